@@ -1,0 +1,110 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention forward library.
+ *
+ * One operation: the chunkwise forward (prefill) pass of Kimi Delta Attention,
+ * i.e. for every sequence and head the recurrence of the Kimi Linear feature
+ * page (chapter 4, "innovation 2", state-update equation)
+ *
+ *     S_t = (Diag(alpha_t) - beta_t k_t (k_t (.) alpha_t)^T) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t,          alpha_t = exp(g_t) per key channel,
+ *
+ * with a 128 x 128 state per head (rows: key channels, columns: value
+ * channels), evaluated in chunks of 64 tokens. The library interface follows
+ * the FlashKDA README summary (GitHub trending page, "kernel API and
+ * constraints"): query, key, value, gate, beta tensors, head dims K = V = 128
+ * only, variable-length packing through cu_seqlens with batch 1, and optional
+ * bf16 or fp32 initial / final states whose dtypes must match when both are
+ * given.
+ *
+ * Conventions for every entry point below:
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device, owned
+ *    by the caller; the library keeps no reference after the call returns.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
+ *    stream) and runs asynchronously: no host synchronisation happens inside.
+ *  - Argument errors are detected before anything is enqueued and returned as
+ *    a kda_status; nothing is written then. Launch failures return
+ *    KDA_ERR_CUDA (the CUDA error is left for cudaGetLastError()).
+ *  - The library allocates no device memory in kda_fwd.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kda_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_NULL_PTR = 1,          /* a required pointer is NULL                         */
+    KDA_ERR_BAD_SHAPE = 2,         /* head dims != 128, negative sizes, H < 1, ...       */
+    KDA_ERR_VARLEN_BATCH = 3,      /* cu_seqlens given with batch != 1                   */
+    KDA_ERR_STATE_DTYPE = 4,       /* state dtype not bf16/fp32, or initial != final     */
+    KDA_ERR_CUDA = 5,              /* a CUDA call failed (launch, attribute, device query) */
+    KDA_ERR_UNSUPPORTED_DEVICE = 6,/* the current device is not sm_100 (B200 class)      */
+    KDA_ERR_BAD_ALIGNMENT = 7,     /* a tensor pointer is not 16-byte aligned            */
+    KDA_ERR_TOO_LARGE = 8          /* sizes exceed what the library indexes              */
+} kda_status;
+
+typedef enum { KDA_DTYPE_NONE = 0, KDA_DTYPE_BF16 = 1, KDA_DTYPE_FP32 = 2 } kda_dtype;
+
+/*
+ * kda_fwd -- chunkwise KDA forward over a batch of independent sequences.
+ *
+ * Layouts (row-major, innermost last, all contiguous):
+ *   q, k, v  : bf16  [batch, seq_len, num_heads, 128]
+ *   g        : fp32  [batch, seq_len, num_heads, 128]  log alpha, raw per token
+ *              (not cumulative); the kernel applies no activation to it
+ *   beta     : fp32  [batch, seq_len, num_heads]
+ *   out      : bf16  [batch, seq_len, num_heads, 128]  (written)
+ *   initial_state, final_state : [num_seqs_eff, num_heads, 128 (key), 128 (value)],
+ *              value index fastest, dtype initial_dtype / final_dtype.
+ * q and k are used as given (the kernel does not normalise them).
+ *
+ * Sequences:
+ *   cu_seqlens == NULL : num_seqs_eff = batch, sequence b is row b (seq_len tokens).
+ *   cu_seqlens != NULL : batch must be 1; cu_seqlens is a DEVICE int32 array of
+ *                        num_seqs + 1 offsets into the seq_len packed tokens,
+ *                        cu_seqlens[0] = 0, non-decreasing, last = seq_len;
+ *                        num_seqs_eff = num_seqs. Entries are clamped into
+ *                        [0, seq_len] and a decreasing pair is read as an empty
+ *                        sequence, so a malformed table cannot make the kernel
+ *                        access memory out of bounds (its results are then
+ *                        unspecified). Zero-length sequences are allowed: their
+ *                        final state equals their initial state.
+ *
+ * State:
+ *   initial_state == NULL (initial_dtype ignored) means zero initial states.
+ *   final_state   == NULL (final_dtype ignored) means the final states are not
+ *   written. A given state must be KDA_DTYPE_BF16 or KDA_DTYPE_FP32 and, when
+ *   both are given, the two dtypes must be equal. The state is carried in fp32
+ *   inside the kernel; a bf16 final state is rounded to nearest even.
+ *
+ * scale multiplies the output (o_t = scale * S_t^T q_t); callers normally
+ * pass 1/sqrt(128).
+ *
+ * head_dim_k and head_dim_v must both be 128. All tensor pointers must be
+ * 16-byte aligned (cu_seqlens 4-byte). Returns KDA_OK once the work is
+ * enqueued.
+ */
+kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, float scale, const int32_t *cu_seqlens,
+                   int32_t num_seqs, int32_t batch, int64_t seq_len, int32_t num_heads,
+                   int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
+                   kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype,
+                   void *out, kda_stream_t stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *kda_status_string(kda_status status);
+
+/* Library ABI version, (major << 16) | minor. */
+int32_t kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,94 @@
+// kda_api.cu -- C-ABI front end: argument validation and kernel dispatch.
+#include <cuda_runtime.h>
+
+#include "../../include/kda.h"
+#include "kda_internal.h"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool device_is_sm100(int *err) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { *err = 1; return false; }
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+        *err = 1;
+        return false;
+    }
+    *err = 0;
+    return major == 10;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_NULL_PTR: return "KDA_ERR_NULL_PTR: a required pointer is NULL";
+        case KDA_ERR_BAD_SHAPE: return "KDA_ERR_BAD_SHAPE: head dims must be 128 and sizes non-negative";
+        case KDA_ERR_VARLEN_BATCH: return "KDA_ERR_VARLEN_BATCH: cu_seqlens requires batch == 1";
+        case KDA_ERR_STATE_DTYPE: return "KDA_ERR_STATE_DTYPE: states must be bf16 or fp32 and match";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call failed";
+        case KDA_ERR_UNSUPPORTED_DEVICE: return "KDA_ERR_UNSUPPORTED_DEVICE: needs an sm_100 (B200) device";
+        case KDA_ERR_BAD_ALIGNMENT: return "KDA_ERR_BAD_ALIGNMENT: tensor pointers must be 16-byte aligned";
+        case KDA_ERR_TOO_LARGE: return "KDA_ERR_TOO_LARGE: sizes exceed the library's index range";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+int32_t kda_version(void) { return (1 << 16) | 0; }
+
+kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, float scale, const int32_t *cu_seqlens,
+                   int32_t num_seqs, int32_t batch, int64_t seq_len, int32_t num_heads,
+                   int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
+                   kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype,
+                   void *out, kda_stream_t stream) {
+    if (head_dim_k != kda::kHeadDim || head_dim_v != kda::kHeadDim) return KDA_ERR_BAD_SHAPE;
+    if (batch < 0 || seq_len < 0 || num_heads < 1 || num_seqs < 0) return KDA_ERR_BAD_SHAPE;
+    if (cu_seqlens && batch != 1) return KDA_ERR_VARLEN_BATCH;
+    if (initial_state && initial_dtype != KDA_DTYPE_BF16 && initial_dtype != KDA_DTYPE_FP32)
+        return KDA_ERR_STATE_DTYPE;
+    if (final_state && final_dtype != KDA_DTYPE_BF16 && final_dtype != KDA_DTYPE_FP32)
+        return KDA_ERR_STATE_DTYPE;
+    if (initial_state && final_state && initial_dtype != final_dtype) return KDA_ERR_STATE_DTYPE;
+    const int64_t n_seqs = cu_seqlens ? num_seqs : batch;
+    const int64_t rows = cu_seqlens ? seq_len : static_cast<int64_t>(batch) * seq_len;
+    if (rows > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL_PTR;
+    if (cu_seqlens && !(reinterpret_cast<uintptr_t>(cu_seqlens) % 4 == 0)) return KDA_ERR_BAD_ALIGNMENT;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(out) ||
+        !aligned16(initial_state) || !aligned16(final_state) ||
+        (reinterpret_cast<uintptr_t>(beta) & 3u))
+        return KDA_ERR_BAD_ALIGNMENT;
+    // token offsets are formed as (row * H + h) * 128 in 64-bit; keep the product well inside
+    if (rows > (int64_t(1) << 40) / (int64_t(num_heads) * kda::kHeadDim)) return KDA_ERR_TOO_LARGE;
+    if (n_seqs * num_heads > (int64_t(1) << 29)) return KDA_ERR_TOO_LARGE;
+    if (n_seqs == 0) return KDA_OK;
+
+    int qerr = 0;
+    if (!device_is_sm100(&qerr)) return qerr ? KDA_ERR_CUDA : KDA_ERR_UNSUPPORTED_DEVICE;
+
+    kda::FwdParams p;
+    p.q = static_cast<const uint16_t *>(q);
+    p.k = static_cast<const uint16_t *>(k);
+    p.v = static_cast<const uint16_t *>(v);
+    p.g = g;
+    p.beta = beta;
+    p.scale = scale;
+    p.cu_seqlens = cu_seqlens;
+    p.seq_len = seq_len;
+    p.num_seqs = static_cast<int32_t>(n_seqs);
+    p.num_heads = num_heads;
+    p.h0 = initial_state;
+    p.h0_fp32 = initial_dtype == KDA_DTYPE_FP32;
+    p.hT = final_state;
+    p.hT_fp32 = final_dtype == KDA_DTYPE_FP32;
+    p.out = static_cast<uint16_t *>(out);
+    const cudaError_t err = kda::launch_fwd_simt(p, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"
