@@ -250,7 +250,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=4096,
                     help="tokens (all heads) in the oracle's CPU-baseline sample")
-    ap.add_argument("--ref-tokens", type=int, default=1024,
+    ap.add_argument("--ref-tokens", type=int, default=8192,
                     help="tokens (all heads) per reference-arm step")
     ap.add_argument("--e2e-slice", type=int, default=1 << 16,
                     help="tokens per host->device slice in the end-to-end measurement")
@@ -329,8 +329,15 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r = cpu_baseline_run(inp, args.cpu_tokens)
+        # size the sample for roughly 10-30 s of host work: probe, then scale up
+        ntok = min(args.cpu_tokens, tokens)
+        r = cpu_baseline_run(inp, ntok)
         secs = r["seconds"][0]
+        if secs < 8.0 and ntok < tokens:
+            ntok = int(min(tokens, ntok * max(1.0, 12.0 / max(secs, 1e-3))))
+            ntok = max(64, ntok // 64 * 64)
+            r = cpu_baseline_run(inp, ntok)
+            secs = r["seconds"][0]
         cpu = {"value": r["tokens"] / secs, "unit": "tokens/s", "cores": r["threads"],
                "kind": "oracle",
                "sample": f"first {r['tokens']} tokens of all {r['heads']} heads of the workload "
