@@ -46,7 +46,8 @@ typedef enum {
     KDA_ERR_CUDA = 5,              /* a CUDA call failed (launch, attribute, device query) */
     KDA_ERR_UNSUPPORTED_DEVICE = 6,/* the current device is not sm_100 (B200 class)      */
     KDA_ERR_BAD_ALIGNMENT = 7,     /* a tensor pointer is not 16-byte aligned            */
-    KDA_ERR_TOO_LARGE = 8          /* sizes exceed what the library indexes              */
+    KDA_ERR_TOO_LARGE = 8,         /* sizes exceed what the library indexes              */
+    KDA_ERR_TIMEOUT = 9            /* a kernel gave up on a bounded wait (see kda_device_error) */
 } kda_status;
 
 typedef enum { KDA_DTYPE_NONE = 0, KDA_DTYPE_BF16 = 1, KDA_DTYPE_FP32 = 2 } kda_dtype;
@@ -96,6 +97,16 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
                    int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
                    kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype,
                    void *out, kda_stream_t stream);
+
+/*
+ * kda_device_error -- synchronise the current device, then read and clear the
+ * library's device-side error word. Every wait inside the kernels is bounded
+ * (a few seconds); a kernel that gives up raises this word and returns early
+ * instead of hanging, leaving its outputs unspecified. Returns KDA_ERR_TIMEOUT
+ * if that happened on this device since the previous call, KDA_OK otherwise,
+ * KDA_ERR_CUDA if the device could not be synchronised or read.
+ */
+kda_status kda_device_error(void);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *kda_status_string(kda_status status);

@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libkda.so")
 
 # entry points declared in include/kda.h
-EXPORTS = ("kda_fwd", "kda_status_string", "kda_version")
+EXPORTS = ("kda_device_error", "kda_fwd", "kda_status_string", "kda_version")
 
 KDA_DTYPE_NONE, KDA_DTYPE_BF16, KDA_DTYPE_FP32 = 0, 1, 2
 
@@ -51,9 +51,16 @@ def load_library(path: str | None = None):
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_version.restype = ctypes.c_int32
         lib.kda_version.argtypes = []
+        lib.kda_device_error.restype = ctypes.c_int
+        lib.kda_device_error.argtypes = []
         if path is None:
             _lib = lib
         return lib
+
+
+def device_error() -> int:
+    """Synchronise and read/clear the device-side error word (0 = no kernel gave up)."""
+    return int(load_library().kda_device_error())
 
 
 def status_string(status: int) -> str:

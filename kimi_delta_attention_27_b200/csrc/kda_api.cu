@@ -35,6 +35,7 @@ const char *kda_status_string(kda_status s) {
         case KDA_ERR_UNSUPPORTED_DEVICE: return "KDA_ERR_UNSUPPORTED_DEVICE: needs an sm_100 (B200) device";
         case KDA_ERR_BAD_ALIGNMENT: return "KDA_ERR_BAD_ALIGNMENT: tensor pointers must be 16-byte aligned";
         case KDA_ERR_TOO_LARGE: return "KDA_ERR_TOO_LARGE: sizes exceed the library's index range";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a kernel gave up waiting on a barrier and stopped";
     }
     return "KDA_ERR_UNKNOWN";
 }
@@ -87,8 +88,15 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
     p.hT = final_state;
     p.hT_fp32 = final_dtype == KDA_DTYPE_FP32;
     p.out = static_cast<uint16_t *>(out);
-    const cudaError_t err = kda::launch_fwd_simt(p, reinterpret_cast<cudaStream_t>(stream));
+    const cudaError_t err = kda::launch_fwd_tc(p, rows, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_device_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return KDA_ERR_CUDA;
+    unsigned int v = 0;
+    if (kda::read_and_clear_device_error(&v) != cudaSuccess) return KDA_ERR_CUDA;
+    return v ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 
 }  // extern "C"

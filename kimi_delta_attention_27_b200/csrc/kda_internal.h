@@ -28,4 +28,11 @@ struct FwdParams {
 // First, straightforward CUDA-core path (fp32 arithmetic throughout).
 cudaError_t launch_fwd_simt(const FwdParams &p, cudaStream_t stream);
 
+// Tensor-core path: one 4-CTA cluster per (sequence, head); `rows` is the
+// number of token rows of the packed [rows, H, 128] tensors.
+cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream);
+
+// Device-side error word of the tensor-core kernel (bit 0: a bounded wait gave up).
+cudaError_t read_and_clear_device_error(unsigned int *value);
+
 }  // namespace kda
