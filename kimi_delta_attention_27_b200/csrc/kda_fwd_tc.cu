@@ -45,6 +45,22 @@ namespace kda {
 
 __device__ unsigned int g_kda_device_error = 0;
 
+#ifdef KDA_TRACE
+// Development-only timeline: when built with -DKDA_TRACE, the first cluster
+// records %globaltimer at fixed points per chunk into g_kda_trace
+// [rank][chunk < 64][point < 16]. The product build compiles none of this.
+__device__ unsigned long long g_kda_trace[4 * 64 * 16];
+#define KDA_TRACE_POINT(chunk, point)                                                               \
+    do {                                                                                            \
+        if (blockIdx.x < 4 && (chunk) < 64)                                                         \
+            g_kda_trace[(rank * 64 + (chunk)) * 16 + (point)] = ptx::globaltimer();                 \
+    } while (0)
+#else
+#define KDA_TRACE_POINT(chunk, point) \
+    do {                              \
+    } while (0)
+#endif
+
 namespace tc {
 
 using namespace ptx;
@@ -259,6 +275,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int sl = n & 1, b = n & 1;
             const uint32_t slot = sbase + sl * SLOT_BYTES;
             if (!wait_bar(BAR(B_SLOT_FULL + sl), (n >> 1) & 1, abort_flag)) break;
+            if (lane == 0) KDA_TRACE_POINT(n, 12);
             if (!wait_bar(BAR(B_VCONV + b), (n >> 1) & 1, abort_flag)) break;
             if (n >= 1 && !wait_bar(BAR(B_C1_FREE), (n - 1) & 1, abort_flag)) break;
             tc_fence_after();
@@ -273,6 +290,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             __syncwarp();
             if (!wait_bar(BAR(B_S_READY), n & 1, abort_flag)) break;
             tc_fence_after();
+            if (lane == 0) KDA_TRACE_POINT(n, 13);
             if (lane == 0) {
                 // state part: [-W; Qt] * S'   (bf16)
                 for (int ks = 0; ks < 8; ++ks)
@@ -400,6 +418,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
             if (!wait_bar(BAR(B_C1_FULL), n & 1, abort_flag)) break;
             tc_fence_after();
+            if (t == 0) KDA_TRACE_POINT(n, 9);
             uint32_t r[32];
             tmem_ld32(tmem + lane_base + COL_C1, r);
             tmem_wait_ld();
@@ -438,6 +457,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (n + 1 < nch && !convert_v(n + 1)) break;
             if (!wait_bar(BAR(B_C3_FULL), n & 1, abort_flag)) break;
             tc_fence_after();
+            if (t == 0) KDA_TRACE_POINT(n, 10);
             tmem_ld32(tmem + lane_base + COL_C3, r);
             tmem_wait_ld();
             const float dec = reinterpret_cast<const float *>(sgen + OFF_DEC + sl * DEC_BYTES)[t];
@@ -452,6 +472,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (lane == 0 && n + 1 < nch) mbar_arrive(BAR(B_S_READY));
             // hand slot `sl` on to the producer of chunk n + 2 once all four warps are done with it
             named_bar_sync(1, 128);
+            if (t == 0) KDA_TRACE_POINT(n, 11);
             if (t == 0 && n + 2 < nch) {
                 const uint32_t prod = static_cast<uint32_t>((n + 2) % NS);
                 if (prod != rank) mbar_expect_tx(BAR(B_SLOT_FULL + sl), SLOT_TX);
@@ -490,9 +511,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int j = static_cast<int>(rank) >= 2 ? kk : kk - 1;
                 if (!wait_bar(BAR(B_SLOT_EMPTY + sl), j & 1, abort_flag)) break;
             }
+            if (t == 0) KDA_TRACE_POINT(m, 0);
             if (t < C) beta_s[t] = t < L ? p.beta[(t0 + t) * H + h] : 0.f;
             if (!wait_bar(BAR(B_STAGE_FULL), kk & 1, abort_flag)) break;
             named_bar_sync(2, 128);
+            if (t == 0) KDA_TRACE_POINT(m, 1);
 
             // -------- S1: running log-decay of channel t, decayed factors (T-format tiles)
             {
@@ -544,11 +567,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             fence_proxy_async_smem();
             named_bar_sync(2, 128);
-            if (t == 0) mbar_arrive(BAR(B_EW_DONE));
+            if (t == 0) { mbar_arrive(BAR(B_EW_DONE)); KDA_TRACE_POINT(m, 2); }
 
             // -------- S2 epilogue: A (fp32, masked, beta-scaled) and Aqk (fp16 + bf16)
             if (!wait_bar(BAR(B_P1_DONE), kk & 1, abort_flag)) break;
             tc_fence_after();
+            if (t == 0) KDA_TRACE_POINT(m, 3);
             {
                 uint32_t a0[32], a1[32];
                 tmem_ld32(tmem + lane_base + COL_P1, a0);
@@ -659,11 +683,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             fence_proxy_async_smem();
             named_bar_sync(2, 128);
-            if (t == 0) mbar_arrive(BAR(B_SOLVE_DONE));
+            if (t == 0) { mbar_arrive(BAR(B_SOLVE_DONE)); KDA_TRACE_POINT(m, 4); }
 
             // -------- S4 epilogues: W (anchored copy + final negated/unanchored), Aqk T'
             if (!wait_bar(BAR(B_WAV_DONE), kk & 1, abort_flag)) break;
             tc_fence_after();
+            if (t == 0) KDA_TRACE_POINT(m, 5);
             {
                 uint32_t a0[32], a1[32];
                 tmem_ld32(tmem + lane_base + COL_W, a0);
@@ -699,11 +724,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar_sync(2, 128);
-            if (t == 0) mbar_arrive(BAR(B_WEPI_DONE));
+            if (t == 0) { mbar_arrive(BAR(B_WEPI_DONE)); KDA_TRACE_POINT(m, 6); }
 
             // -------- Qt = (Qh - Aqk W') e^Ga, row t of Qt^T, in place over Qh^T
             if (!wait_bar(BAR(B_Q_DONE), kk & 1, abort_flag)) break;
             tc_fence_after();
+            if (t == 0) KDA_TRACE_POINT(m, 7);
             {
                 uint32_t a0[32], a1[32];
                 tmem_ld32(tmem + lane_base + COL_Q, a0);
@@ -742,6 +768,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     mbar_arrive_remote(rfull);
                 }
                 mbar_arrive(full);
+                KDA_TRACE_POINT(m, 8);
             }
         }
     }
@@ -833,6 +860,12 @@ cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream)
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
+
+#ifdef KDA_TRACE
+extern "C" int kda_trace_read(unsigned long long *host) {
+    return static_cast<int>(cudaMemcpyFromSymbol(host, g_kda_trace, sizeof(g_kda_trace)));
+}
+#endif
 
 cudaError_t read_and_clear_device_error(unsigned int *value) {
     cudaError_t err = cudaMemcpyFromSymbol(value, g_kda_device_error, sizeof(unsigned int));
