@@ -11,32 +11,37 @@
 //   Akk = strict_lower(diag(beta) Akk_raw), Aqk = lower(Aqk)
 //   T' = (I + Akk)^-1 diag(beta)                            (S3, blocked substitution)
 //   W' = T' Kh;  W = W' diag(e^Ga)                          (S4)
-//   Qt = (Qh - Aqk W') diag(e^Ga)                           (output read-out folded with the
+//   Qt = (Qh - Aqk W') diag(e^Ga)                           (read-out folded with the
 //                                                            intra-chunk attention)
-//   AV = [T'; Aqk T']                                       (S4, value side)
-//   X  = [-W; Qt] S + AV V        ->  X[0:64] = D (pseudo-values), X[64:128] = O / scale   (S5 + S6)
+//   UV = [T'; Aqk T'] V = [U; Aqk U]                        (S4, value side)
+//   X  = [-W; Qt] S + UV      ->  X[0:64] = D (pseudo-values), X[64:128] = O / scale (S5+S6)
 //   S <- diag(e^Gl) S + Kt^T D                              (S7)
 //
-// Layout on the GPU: one cluster of 4 CTAs per (sequence, head); CTA r owns value
-// columns [32 r, 32 r + 32) of the state, its output slice and the state-dependent
-// chain (S5-S7) for them. The state-independent work of a chunk (S1-S4) depends on
-// q, k, g, beta only, so chunk n is prepared by CTA n % 4 alone, which then pushes
-// the finished operand tiles (64.5 KB) into a slot of every CTA's shared memory by
-// bulk copies; each CTA reads q, k, g for a quarter of the chunks and v for its own
-// slice, so every input byte crosses HBM once.
-//
-// Warp roles (384 threads): w0 value-slice TMA, w1 chain MMA issuer, w2 prep MMA
-// issuer, w3 prep TMA, w4-7 chain epilogue (TMEM lanes = state rows / chunk rows),
-// w8-11 chunk preparation (elementwise gates, UT solve, epilogues).
+// Work split: one 4-CTA cluster per (sequence, head).
+//  * rank 0 ("chain") owns the whole fp32 state (128 x 128) and runs the sequential
+//    part, S5-S7, with 128-column MMAs: the dependent-step latency of a tcgen05 MMA
+//    is the same for N = 32 and N = 128, so the state is not split.
+//  * ranks 1-3 ("prep") each prepare every third chunk (S0-S4: gates, decayed
+//    blocks, UT solve, W / Qt / Kt and the value side UV), writing the finished
+//    80.5 KB operand set
+//    into a per-cluster ring of 6 slots in global memory (it stays in L2); the
+//    chain CTA pulls each set with one TMA bulk load. Shared memory of another
+//    CTA (DSMEM) carries only barrier signals: its bulk bandwidth is a fraction
+//    of an L2 TMA load's.
+//  Every input byte is read from HBM once (q, k, v, g, beta by a prep CTA) and
+//  every output byte written once (by the chain CTA).
 //
 // Precision: anchored factors (Kh, Qh, Kc), W, Qt and the state copy S' are bf16;
-// T', AV, the value slice, Kt and D are fp16 (10-bit mantissa) because the state
-// update is most sensitive to them; every product accumulates in fp32 (TMEM) and the
-// state itself is carried in fp32 registers.
+// T', Aqk T', V, UV, Kt and D are fp16 (10-bit mantissa) because the state update is
+// most sensitive to them; every product accumulates in fp32 (TMEM) and the state itself
+// is carried in fp32 registers.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
 
 #include "kda_internal.h"
 #include "sm100_ptx.cuh"
@@ -67,63 +72,91 @@ using namespace ptx;
 
 constexpr int D = kHeadDim;
 constexpr int C = kChunk;
-constexpr int NS = 4;          // CTAs per cluster = value slices
-constexpr int NV = D / NS;     // 32 value columns per CTA
+constexpr int NS = 4;          // CTAs per cluster: 1 chain + 3 prep
+constexpr int NPREP = NS - 1;
 constexpr int NTHREADS = 384;
-constexpr int ANCHOR = 31;
+constexpr int NRING = 6;       // ring slots per cluster (multiple of NPREP)
 
-// ---- shared memory map (byte offsets from a 1024-aligned base)
-constexpr uint32_t SLOT_BYTES = 65536;
-constexpr uint32_t SLOT_KT = 0, SLOT_W = 16384, SLOT_Q = 32768, SLOT_AV = 49152;
-constexpr uint32_t OFF_DEC = 2 * SLOT_BYTES;       // e^Gl per slot, 128 fp32
-constexpr uint32_t DEC_BYTES = 512;
-constexpr uint32_t SLOT_TX = 4 * 16384 + DEC_BYTES;
-constexpr uint32_t OFF_STAGE = OFF_DEC + 1024;     // q, k, g staging; then UT workspace
-constexpr uint32_t STG_Q = 0, STG_K = 16384, STG_G = 32768, STAGE_TX = 65536;
-constexpr uint32_t AKK_LD = 68;                    // fp32 row stride (floats) of A and T
-constexpr uint32_t WS_AKK = 0, WS_T = 17408, WS_P = 34816, WS_TB = 0, WS_AQB = 40960, WS_WP = 49152;
-constexpr uint32_t OFF_SP = OFF_STAGE + 65536;     // S' [128 x 32] bf16, MN-major SW64
-constexpr uint32_t OFF_DL = OFF_SP + 8192;         // D  [64 x 32] fp16, MN-major SW64
-constexpr uint32_t OFF_V = OFF_DL + 4096;          // V  2 x [64 x 32], SW64
-constexpr uint32_t OFF_MISC = OFF_V + 8192;
-constexpr uint32_t OFF_BAR = OFF_MISC;             // 32 mbarriers
-constexpr uint32_t OFF_BETA = OFF_BAR + 256;       // 64 fp32
-constexpr uint32_t OFF_EGA = OFF_BETA + 256;       // 128 fp32
-constexpr uint32_t OFF_TMEMPTR = OFF_EGA + 512;
-constexpr uint32_t OFF_ABORT = OFF_TMEMPTR + 16;
-constexpr uint32_t SMEM_USED = OFF_ABORT + 16;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+// ---- operand set of one chunk (same byte layout in the global ring and in smem)
+//   Kt^T fp16 [128 x 64] | -W^T bf16 [128 x 64] | Qt^T bf16 [128 x 64] |
+//   UV fp16 [128 x 128] as two 64-column blocks | e^Gl fp32 [128]
+constexpr uint32_t SET_KT = 0, SET_W = 16384, SET_Q = 32768, SET_UV = 49152, SET_DEC = 81920;
+constexpr uint32_t SET_BYTES = SET_DEC + 512;      // 82432
+constexpr uint32_t SET_STRIDE = 83968;             // 82 KB, 1024-aligned
+constexpr uint64_t RING_BYTES = static_cast<uint64_t>(NRING) * SET_STRIDE;
+constexpr int kMaxRings = 256;                     // indexed by the chain CTA's SM id
 
-// barrier indices
+// ---- chain CTA shared memory
+constexpr uint32_t CH_SLOT = 0;                    // 2 x SET_STRIDE
+constexpr uint32_t CH_SP = 2 * SET_STRIDE;         // S' [128 x 128] bf16 MN-major SW128 (two 16 KB blocks)
+constexpr uint32_t CH_DL = CH_SP + 32768;          // D  [64 x 128] fp16 MN-major SW128 (two 8 KB blocks)
+constexpr uint32_t CH_MISC = CH_DL + 16384;
+// ---- prep CTA shared memory
+constexpr uint32_t PR_STG = 0;                     // q 16 KB, k 16 KB, g 32 KB, v 16 KB
+constexpr uint32_t STG_Q = 0, STG_K = 16384, STG_G = 32768, STG_V = 65536, STAGE_TX = 65536, VSTAGE_TX = 16384;
+constexpr uint32_t PR_KH = 81920, PR_QH = PR_KH + 16384, PR_KC = PR_QH + 16384;
+constexpr uint32_t AKK_LD = 68;                    // fp32 row stride of A and T
+constexpr uint32_t PR_AKK = PR_KC + 16384;         // 17408 B
+constexpr uint32_t PR_T = PR_AKK + 17408;          // 17408 B
+constexpr uint32_t PR_P = PR_T + 17408;            // 4096 B
+constexpr uint32_t PR_AVT = 169984;                // [T'h; (Aqk T')_h] fp16, 128 rows K-major SW128
+constexpr uint32_t PR_TB = PR_AVT + 16384;         // T' bf16
+constexpr uint32_t PR_AQB = PR_TB + 8192;          // Aqk bf16
+constexpr uint32_t PR_WP = PR_AQB + 8192;          // W'^T bf16
+constexpr uint32_t PR_MISC = PR_WP + 16384;
+static_assert(PR_P + 4096 <= PR_AVT, "prep map");
+static_assert(PR_AVT % 1024 == 0 && PR_WP % 1024 == 0 && CH_SP % 1024 == 0 && PR_KH % 1024 == 0, "alignment");
+
+// misc area (offsets from the misc base of either role)
+constexpr uint32_t M_BAR = 0;                      // up to 32 barriers
+constexpr uint32_t M_BETA = 256, M_EGA = 512, M_GSUM = 1024;   // 64, 128, 2 x 128 floats
+constexpr uint32_t M_DEC = 2048;                               // 2 x 128 floats (e^Gl, part of the set)
+constexpr uint32_t M_TMEM = 3072, M_ABORT = 3088, M_SMID = 3104;
+constexpr uint32_t MISC_BYTES = 3584;
+constexpr uint32_t SMEM_USED = (CH_MISC > PR_MISC ? CH_MISC : PR_MISC) + MISC_BYTES;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
+
+// chain barriers
 enum {
-    B_SLOT_FULL = 0,   // 2
-    B_SLOT_EMPTY = 2,  // 2
-    B_VFULL = 4,       // 2
-    B_VCONV = 6,       // 2
-    B_VFREE = 8,       // 2
-    B_C1_FULL = 10, B_C1_FREE, B_S_READY, B_D_READY, B_C3_FULL,
-    B_STAGE_FULL, B_STAGE_FREE, B_EW_DONE, B_P1_DONE, B_SOLVE_DONE, B_WAV_DONE, B_WEPI_DONE, B_Q_DONE,
-    B_COUNT
+    CB_FULL = 0,     // 2: operand set landed in smem slot (1 arrival + tx)
+    CB_SFREE = 2,    // 2: smem slot consumed (8 epilogue warps + the output store warp)
+    CB_C1_FULL = 4, CB_C1_FREE, CB_S_READY, CB_D_READY, CB_C3_FULL,
+    CB_O_READY = 9,  // output tile staged in the slot (4 warps)
+    CB_READY = 10,   // 6: ring slot written by a prep CTA (remote arrival)
+    CB_COUNT = 16
 };
-static_assert(B_COUNT * 8 <= 256, "barrier area");
+// prep barriers
+enum {
+    PB_STAGE_FULL = 0, PB_STAGE_FREE, PB_VSTAGE_FULL, PB_VSTAGE_FREE, PB_EW_DONE, PB_P1_DONE, PB_SOLVE_DONE,
+    PB_WAV_DONE, PB_WEPI_DONE, PB_Q_DONE,
+    PB_OUTA_READY,      // Kt^T final (over Kc^T)
+    PB_OUTB_READY,      // -W^T final (over Kh^T)
+    PB_OUTC_READY,      // Qt^T (over the AV operand), UV (over A / T), e^Gl final
+    PB_OUTAB_FREE,      // publisher has read parts A and B out
+    PB_OUTC_FREE,       // publisher has read part C out
+    PB_RING_FREE = 15,  // 6: ring slot released by the chain CTA (remote arrival)
+    PB_COUNT = 21
+};
+static_assert(CB_COUNT * 8 <= M_BETA && PB_COUNT * 8 <= M_BETA, "barrier area");
 
 // ---- TMEM columns
-constexpr uint32_t COL_P1 = 0, COL_W = 64, COL_AV = 128, COL_Q = 192, COL_C1 = 256, COL_C3 = 288;
+constexpr uint32_t COL_C1 = 0, COL_C3 = 128;                                      // chain
+constexpr uint32_t COL_P1 = 0, COL_W = 64, COL_AV = 128, COL_Q = 192, COL_UV = 256;  // prep
 constexpr uint32_t TMEM_COLS = 512;
 
 // ---- instruction descriptors (M = 128)
-constexpr uint32_t ID_P1 = idesc_f16(128, 64, 1, 1, 1);     // bf16, A MN-major, B MN-major
-constexpr uint32_t ID_W = idesc_f16(128, 64, 1, 0, 0);      // bf16, K-major / K-major
-constexpr uint32_t ID_AV = idesc_f16(128, 64, 0, 0, 1);     // fp16, K-major / MN-major
-constexpr uint32_t ID_Q = idesc_f16(128, 64, 1, 0, 0);      // bf16
-constexpr uint32_t ID_VPART = idesc_f16(128, NV, 0, 0, 1);  // fp16, A K-major, B MN-major
-constexpr uint32_t ID_STATE = idesc_f16(128, NV, 1, 1, 1);  // bf16, A MN-major, B MN-major
-constexpr uint32_t ID_C3 = idesc_f16(128, NV, 0, 0, 1);     // fp16
+constexpr uint32_t ID_P1 = idesc_f16(128, 64, 1, 1, 1);      // bf16, A MN-major, B MN-major
+constexpr uint32_t ID_W = idesc_f16(128, 64, 1, 0, 0);       // bf16, K-major / K-major
+constexpr uint32_t ID_AV = idesc_f16(128, 64, 0, 0, 1);      // fp16, K-major / MN-major
+constexpr uint32_t ID_Q = idesc_f16(128, 64, 1, 0, 0);       // bf16
+constexpr uint32_t ID_UV = idesc_f16(128, 128, 0, 0, 1);     // fp16, A K-major, B MN-major
+constexpr uint32_t ID_STATE = idesc_f16(128, 128, 1, 1, 1);  // bf16, A MN-major, B MN-major
+constexpr uint32_t ID_C3 = idesc_f16(128, 128, 0, 0, 1);     // fp16
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 
 struct TmaMaps {
-    CUtensorMap q, k, g, v;
+    CUtensorMap q, k, g, v, o;
 };
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t *abort_flag) {
@@ -141,6 +174,8 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 }
 
 __device__ __forceinline__ float bf2f(uint16_t x) { return __uint_as_float(static_cast<uint32_t>(x) << 16); }
+__device__ __forceinline__ float lo_bf(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_bf(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -153,8 +188,6 @@ __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
 
 // byte offset of 16-byte chunk j of row r in a tile of 128-byte rows, 128B swizzle
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t j) { return r * 128u + ((j ^ (r & 7u)) << 4); }
-// byte offset of 16-byte chunk j of row r in a tile of 64-byte rows, 64B swizzle
-__device__ __forceinline__ uint32_t sw64(uint32_t r, uint32_t j) { return r * 64u + ((j ^ ((r >> 1) & 3u)) << 4); }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
@@ -168,21 +201,60 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
                  : "memory");
     return v;
 }
+__device__ __forceinline__ void st_global_v4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// bulk copy global -> this CTA's shared memory, completing tx bytes on a local barrier
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+// bulk copy this CTA's shared memory -> global, tracked by the executing thread's bulk groups
+__device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int32_t c0, int32_t c1, int32_t c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t smid() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+    return r;
+}
 
 __global__ void __launch_bounds__(NTHREADS, 1)
-    kda_fwd_tc_kernel(const FwdParams p, const __grid_constant__ TmaMaps maps) {
+    kda_fwd_tc_kernel(const FwdParams p, const __grid_constant__ TmaMaps maps, unsigned char *rings) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = raw + ((1024u - (raw & 1023u)) & 1023u);
     unsigned char *sgen = smem_raw + (sbase - raw);
-    const uint32_t bar0 = sbase + OFF_BAR;
-    auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
-    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sgen + OFF_ABORT);
-    float *beta_s = reinterpret_cast<float *>(sgen + OFF_BETA);
-    float *ega_s = reinterpret_cast<float *>(sgen + OFF_EGA);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
+    const bool is_chain = rank == 0;
+    const uint32_t misc = sbase + (is_chain ? CH_MISC : PR_MISC);
+    unsigned char *miscg = sgen + (is_chain ? CH_MISC : PR_MISC);
+    auto BAR = [&](int i) -> uint32_t { return misc + M_BAR + 8u * static_cast<uint32_t>(i); };
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(miscg + M_ABORT);
+
     const int H = p.num_heads;
     const int64_t unit = blockIdx.x / NS;
     const int h = static_cast<int>(unit % H);
@@ -199,41 +271,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         eos = bos + p.seq_len;
     }
     const int nch = static_cast<int>((eos - bos + C - 1) / C);
-    const int v0 = static_cast<int>(rank) * NV;
     const size_t state_base = (static_cast<size_t>(s) * H + h) * D * D;
 
     // ---------------------------------------------------------------- setup
     if (tid == 0) {
-        mbar_init(BAR(B_SLOT_FULL + 0), 1);
-        mbar_init(BAR(B_SLOT_FULL + 1), 1);
-        mbar_init(BAR(B_SLOT_EMPTY + 0), NS);
-        mbar_init(BAR(B_SLOT_EMPTY + 1), NS);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(BAR(B_VFULL + b), 1);
-            mbar_init(BAR(B_VCONV + b), 4);
-            mbar_init(BAR(B_VFREE + b), 1);
+        if (is_chain) {
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(BAR(CB_FULL + i), 1);
+                mbar_init(BAR(CB_SFREE + i), 9);
+            }
+            mbar_init(BAR(CB_C1_FULL), 1);
+            mbar_init(BAR(CB_C1_FREE), 8);
+            mbar_init(BAR(CB_S_READY), 8);
+            mbar_init(BAR(CB_D_READY), 4);
+            mbar_init(BAR(CB_C3_FULL), 1);
+            mbar_init(BAR(CB_O_READY), 4);
+            for (int i = 0; i < NRING; ++i) mbar_init(BAR(CB_READY + i), 1);
+            const uint32_t sm = smid();
+            *reinterpret_cast<volatile uint32_t *>(miscg + M_SMID) = sm;
+            *abort_flag = sm < static_cast<uint32_t>(kMaxRings) ? 0u : 1u;
+            if (sm >= static_cast<uint32_t>(kMaxRings)) atomicOr(&g_kda_device_error, 2u);
+        } else {
+            for (int i = 0; i < PB_RING_FREE; ++i) mbar_init(BAR(i), 1);
+            for (int i = 0; i < NRING; ++i) mbar_init(BAR(PB_RING_FREE + i), 1);
+            *abort_flag = 0;
         }
-        mbar_init(BAR(B_C1_FULL), 1);
-        mbar_init(BAR(B_C1_FREE), 4);
-        mbar_init(BAR(B_S_READY), 4);
-        mbar_init(BAR(B_D_READY), 2);
-        mbar_init(BAR(B_C3_FULL), 1);
-        mbar_init(BAR(B_STAGE_FULL), 1);
-        mbar_init(BAR(B_STAGE_FREE), 1);
-        mbar_init(BAR(B_EW_DONE), 1);
-        mbar_init(BAR(B_P1_DONE), 1);
-        mbar_init(BAR(B_SOLVE_DONE), 1);
-        mbar_init(BAR(B_WAV_DONE), 1);
-        mbar_init(BAR(B_WEPI_DONE), 1);
-        mbar_init(BAR(B_Q_DONE), 1);
-        *abort_flag = 0;
         fence_mbar_init();
-        // the first two chunks' slots start free: arm them for the bytes a peer will push
-        for (int n = 0; n < 2 && n < nch; ++n)
-            if (n % NS != static_cast<int>(rank)) mbar_expect_tx(BAR(B_SLOT_FULL + (n & 1)), SLOT_TX);
     }
     if (warp == 2) {
-        tmem_alloc(sbase + OFF_TMEMPTR, TMEM_COLS);
+        tmem_alloc(misc + M_TMEM, TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -241,534 +307,715 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     cluster_arrive();
     cluster_wait();
     tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sgen + OFF_TMEMPTR);
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(miscg + M_TMEM);
+    // this cluster's ring: indexed by the chain CTA's SM (unique among resident clusters)
+    const uint32_t ring_id = is_chain ? *reinterpret_cast<volatile uint32_t *>(miscg + M_SMID)
+                                      : ld_shared_cluster_u32(mapa(sbase + CH_MISC + M_SMID, 0));
+    if (!is_chain && ring_id >= static_cast<uint32_t>(kMaxRings) && tid == 0) *abort_flag = 1;
+    unsigned char *ring = rings + static_cast<uint64_t>(ring_id < kMaxRings ? ring_id : 0) * RING_BYTES;
 
-    if (warp == 0) {
-        // ============================================================ value-slice TMA
-        for (int n = 0; n < nch; ++n) {
-            const int b = n & 1;
-            if (n >= 2 && !wait_bar(BAR(B_VFREE + b), ((n - 2) >> 1) & 1, abort_flag)) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(BAR(B_VFULL + b), 4096);
-                tma_load_3d(sbase + OFF_V + b * 4096, &maps.v, BAR(B_VFULL + b), v0, h,
-                            static_cast<int32_t>(bos + static_cast<int64_t>(n) * C));
-            }
-            __syncwarp();
-        }
-    } else if (warp == 3) {
-        // ============================================================ prep TMA (q, k, g)
-        int kk = 0;
-        for (int m = static_cast<int>(rank); m < nch; m += NS, ++kk) {
-            if (kk >= 1 && !wait_bar(BAR(B_STAGE_FREE), (kk - 1) & 1, abort_flag)) break;
-            if (lane == 0) {
-                const int32_t row = static_cast<int32_t>(bos + static_cast<int64_t>(m) * C);
-                mbar_arrive_expect_tx(BAR(B_STAGE_FULL), STAGE_TX);
-                tma_load_3d(sbase + OFF_STAGE + STG_Q, &maps.q, BAR(B_STAGE_FULL), 0, h, row);
-                tma_load_3d(sbase + OFF_STAGE + STG_K, &maps.k, BAR(B_STAGE_FULL), 0, h, row);
-                tma_load_3d(sbase + OFF_STAGE + STG_G, &maps.g, BAR(B_STAGE_FULL), 0, h, row);
-            }
-            __syncwarp();
-        }
-    } else if (warp == 1) {
-        // ============================================================ chain MMA issuer
-        for (int n = 0; n < nch; ++n) {
-            const int sl = n & 1, b = n & 1;
-            const uint32_t slot = sbase + sl * SLOT_BYTES;
-            if (!wait_bar(BAR(B_SLOT_FULL + sl), (n >> 1) & 1, abort_flag)) break;
-            if (lane == 0) KDA_TRACE_POINT(n, 12);
-            if (!wait_bar(BAR(B_VCONV + b), (n >> 1) & 1, abort_flag)) break;
-            if (n >= 1 && !wait_bar(BAR(B_C1_FREE), (n - 1) & 1, abort_flag)) break;
-            tc_fence_after();
-            if (lane == 0) {
-                // value part: [T'; Aqk T'] * V   (fp16)
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tmem + COL_C1, smem_desc(slot + SLOT_AV + ks * 32, 16, 1024, kSwizzle128),
-                            smem_desc(sbase + OFF_V + b * 4096 + ks * 1024, 4096, 512, kSwizzle64), ID_VPART,
-                            ks > 0);
-                mma_commit(BAR(B_VFREE + b));
-            }
-            __syncwarp();
-            if (!wait_bar(BAR(B_S_READY), n & 1, abort_flag)) break;
-            tc_fence_after();
-            if (lane == 0) KDA_TRACE_POINT(n, 13);
-            if (lane == 0) {
-                // state part: [-W; Qt] * S'   (bf16)
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_f16(tmem + COL_C1, smem_desc(slot + SLOT_W + ks * 2048, 16384, 1024, kSwizzle128),
-                            smem_desc(sbase + OFF_SP + ks * 1024, 4096, 512, kSwizzle64), ID_STATE, 1);
-                mma_commit(BAR(B_C1_FULL));
-            }
-            __syncwarp();
-            if (!wait_bar(BAR(B_D_READY), n & 1, abort_flag)) break;
-            tc_fence_after();
-            if (lane == 0) {
-                // state increment: Kt^T * D   (fp16)
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tmem + COL_C3, smem_desc(slot + SLOT_KT + ks * 32, 16, 1024, kSwizzle128),
-                            smem_desc(sbase + OFF_DL + ks * 1024, 4096, 512, kSwizzle64), ID_C3, ks > 0);
-                mma_commit(BAR(B_C3_FULL));
-            }
-            __syncwarp();
-        }
-    } else if (warp == 2) {
-        // ============================================================ prep MMA issuer
-        int kk = 0;
-        for (int m = static_cast<int>(rank); m < nch; m += NS, ++kk) {
-            const uint32_t slot = sbase + (m & 1) * SLOT_BYTES;
-            const uint32_t ws = sbase + OFF_STAGE;
-            if (!wait_bar(BAR(B_EW_DONE), kk & 1, abort_flag)) break;
-            tc_fence_after();
-            if (lane == 0) {
-                // [Kh; Qh] Kc^T : A = Kh^T | Qh^T (MN-major, 64-row blocks 16 KB apart), B = Kc^T
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_f16(tmem + COL_P1, smem_desc(slot + SLOT_W + ks * 2048, 16384, 1024, kSwizzle128),
-                            smem_desc(slot + SLOT_AV + ks * 2048, 16384, 1024, kSwizzle128), ID_P1, ks > 0);
-                mma_commit(BAR(B_P1_DONE));
-            }
-            __syncwarp();
-            if (!wait_bar(BAR(B_SOLVE_DONE), kk & 1, abort_flag)) break;
-            tc_fence_after();
-            if (lane == 0) {
-                // W'^T = Kh^T T'^T (bf16)
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tmem + COL_W, smem_desc(slot + SLOT_W + ks * 32, 16, 1024, kSwizzle128),
-                            smem_desc(ws + WS_TB + ks * 32, 16, 1024, kSwizzle128), ID_W, ks > 0);
-                // [T'; Aqk] T' (fp16); only rows 64..127 (Aqk T') are used
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tmem + COL_AV, smem_desc(slot + SLOT_AV + ks * 32, 16, 1024, kSwizzle128),
-                            smem_desc(slot + SLOT_AV + ks * 2048, 16384, 1024, kSwizzle128), ID_AV, ks > 0);
-                mma_commit(BAR(B_WAV_DONE));
-            }
-            __syncwarp();
-            if (!wait_bar(BAR(B_WEPI_DONE), kk & 1, abort_flag)) break;
-            tc_fence_after();
-            if (lane == 0) {
-                // W'^T Aqk^T (bf16)
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tmem + COL_Q, smem_desc(ws + WS_WP + ks * 32, 16, 1024, kSwizzle128),
-                            smem_desc(ws + WS_AQB + ks * 32, 16, 1024, kSwizzle128), ID_Q, ks > 0);
-                mma_commit(BAR(B_Q_DONE));
-            }
-            __syncwarp();
-        }
-    } else if (warp < 8) {
-        // ============================================================ chain epilogue (w4..w7)
-        const int t = tid - 128;               // TMEM lane = state row k = chunk row for C1
-        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        float S[NV];
-        if (p.h0) {
-            const size_t off = state_base + static_cast<size_t>(t) * D + v0;
-            if (p.h0_fp32) {
-                const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(p.h0) + off);
-#pragma unroll
-                for (int j = 0; j < NV / 4; ++j) {
-                    float4 x = src[j];
-                    S[4 * j] = x.x; S[4 * j + 1] = x.y; S[4 * j + 2] = x.z; S[4 * j + 3] = x.w;
-                }
-            } else {
-                const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.h0) + off);
-#pragma unroll
-                for (int j = 0; j < NV / 8; ++j) {
-                    uint4 x = src[j];
-                    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        S[8 * j + 2 * e] = __uint_as_float(w[e] << 16);
-                        S[8 * j + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    if (is_chain) {
+        // ======================================================================= chain CTA
+        if (warp == 0) {
+            // ---- output tiles: staged in the slot's value-side rows 64..127 (two 64-column
+            // boxes, 128B swizzle); TMA-stored for full chunks, copied row by row otherwise
+            for (int n = 0; n < nch; ++n) {
+                const int sl = n & 1;
+                const int64_t t0 = bos + static_cast<int64_t>(n) * C;
+                const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
+                const uint32_t stage = sbase + CH_SLOT + sl * SET_STRIDE + SET_UV + 8192;
+                if (!wait_bar(BAR(CB_O_READY), n & 1, abort_flag)) break;
+                if (L == C) {
+                    if (lane == 0) {
+                        tma_store_3d(&maps.o, stage, 0, h, static_cast<int32_t>(t0));
+                        tma_store_3d(&maps.o, stage + 16384, 64, h, static_cast<int32_t>(t0));
+                        bulk_commit();
+                        bulk_wait_read0();
+                    }
+                } else {
+                    // partial chunk: rows < L only, 16 bytes per lane, a row is 2 x 8 chunks
+                    for (int e = lane; e < L * 16; e += 32) {
+                        const int rr = e >> 4, hb = (e >> 3) & 1, j = e & 7;
+                        const uint4 v = ld_shared_v4(stage + hb * 16384 + sw128(rr, j));
+                        st_global_v4(p.out + ((t0 + rr) * H + h) * D + hb * 64 + j * 8, v.x, v.y, v.z, v.w);
                     }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(BAR(CB_SFREE + sl));
             }
-        } else {
-#pragma unroll
-            for (int j = 0; j < NV; ++j) S[j] = 0.f;
-        }
-        auto write_sprime = [&]() {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                st_shared_v4(sbase + OFF_SP + sw64(t, j), pack_bf16(S[8 * j], S[8 * j + 1]),
-                             pack_bf16(S[8 * j + 2], S[8 * j + 3]), pack_bf16(S[8 * j + 4], S[8 * j + 5]),
-                             pack_bf16(S[8 * j + 6], S[8 * j + 7]));
-        };
-        auto convert_v = [&](int n) -> bool {
-            const int b = n & 1;
-            if (!wait_bar(BAR(B_VFULL + b), (n >> 1) & 1, abort_flag)) return false;
-#pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                const uint32_t a = sbase + OFF_V + b * 4096 + (t + 128 * c2) * 16;
-                uint4 x = ld_shared_v4(a);
-                uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    w[e] = pack_f16(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
-                st_shared_v4(a, w[0], w[1], w[2], w[3]);
+            if (lane == 0) bulk_wait0();
+            __syncwarp();
+        } else if (warp == 2) {
+            // ---- operand sets: ring slot (global, L2) -> smem slot
+            for (int n = 0; n < nch; ++n) {
+                const int sl = n & 1, r = n % NRING;
+                if (!wait_bar(BAR(CB_READY + r), (n / NRING) & 1, abort_flag)) break;
+                if (n >= 2 && !wait_bar(BAR(CB_SFREE + sl), ((n - 2) >> 1) & 1, abort_flag)) break;
+                if (lane == 0) {
+                    const unsigned char *src = ring + static_cast<uint64_t>(r) * SET_STRIDE;
+                    const uint32_t dst = sbase + CH_SLOT + sl * SET_STRIDE;
+                    mbar_arrive_expect_tx(BAR(CB_FULL + sl), SET_BYTES);
+                    for (uint32_t part = 0; part < 5; ++part)
+                        bulk_g2s(dst + part * 16384, src + part * 16384, 16384, BAR(CB_FULL + sl));
+                    bulk_g2s(dst + SET_DEC, src + SET_DEC, 512, BAR(CB_FULL + sl));
+                }
+                __syncwarp();
             }
+        } else if (warp == 1) {
+            // ---- chain MMA issuer
+            for (int n = 0; n < nch; ++n) {
+                const int sl = n & 1;
+                const uint32_t slot = sbase + CH_SLOT + sl * SET_STRIDE;
+                if (!wait_bar(BAR(CB_FULL + sl), (n >> 1) & 1, abort_flag)) break;
+                if (lane == 0) KDA_TRACE_POINT(n, 12);
+                // the ring slot has been copied out: hand it back to the producer of chunk n + NRING
+                if (lane == 0 && n + NRING < nch) {
+                    const uint32_t prod = 1u + static_cast<uint32_t>(n % NPREP);
+                    mbar_arrive_remote(mapa(sbase + PR_MISC + M_BAR + 8u * (PB_RING_FREE + n % NRING), prod));
+                }
+                if (n >= 1 && !wait_bar(BAR(CB_C1_FREE), (n - 1) & 1, abort_flag)) break;
+                if (!wait_bar(BAR(CB_S_READY), n & 1, abort_flag)) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    KDA_TRACE_POINT(n, 13);
+                    // state part: [-W; Qt] * S'   (bf16)
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_f16(tmem + COL_C1, smem_desc(slot + SET_W + ks * 2048, 16384, 1024, kSwizzle128),
+                                smem_desc(sbase + CH_SP + ks * 2048, 16384, 1024, kSwizzle128), ID_STATE, ks > 0);
+                    mma_commit(BAR(CB_C1_FULL));
+                    KDA_TRACE_POINT(n, 3);
+                }
+                __syncwarp();
+                if (!wait_bar(BAR(CB_D_READY), n & 1, abort_flag)) break;
+                tc_fence_after();
+                if (lane == 0) KDA_TRACE_POINT(n, 4);
+                if (lane == 0) {
+                    // state increment: Kt^T * D   (fp16)
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(tmem + COL_C3, smem_desc(slot + SET_KT + ks * 32, 16, 1024, kSwizzle128),
+                                smem_desc(sbase + CH_DL + ks * 2048, 8192, 1024, kSwizzle128), ID_C3, ks > 0);
+                    mma_commit(BAR(CB_C3_FULL));
+                    KDA_TRACE_POINT(n, 5);
+                }
+                __syncwarp();
+            }
+        } else if (warp >= 4) {
+            // ---- epilogues: 8 warps; a warp covers TMEM lanes 32*(warp%4).. and value columns 64*half..
+            const int q4 = warp & 3, half = (warp - 4) >> 2;
+            const int row = q4 * 32 + lane;            // TMEM lane = state row k / chunk row
+            const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+            const int c0 = half * 64;                  // first value column of this thread
+            float S[64];
+            if (p.h0) {
+                const size_t off = state_base + static_cast<size_t>(row) * D + c0;
+                if (p.h0_fp32) {
+                    const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(p.h0) + off);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float4 x = src[j];
+                        S[4 * j] = x.x; S[4 * j + 1] = x.y; S[4 * j + 2] = x.z; S[4 * j + 3] = x.w;
+                    }
+                } else {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.h0) + off);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 x = src[j];
+                        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            S[8 * j + 2 * e] = lo_bf(w[e]);
+                            S[8 * j + 2 * e + 1] = hi_bf(w[e]);
+                        }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) S[j] = 0.f;
+            }
+            // S' (bf16, MN-major: column block `half`, row `row`)
+            auto write_sprime = [&]() {
+                const uint32_t base = sbase + CH_SP + half * 16384;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    st_shared_v4(base + sw128(row, j), pack_bf16(S[8 * j], S[8 * j + 1]),
+                                 pack_bf16(S[8 * j + 2], S[8 * j + 3]), pack_bf16(S[8 * j + 4], S[8 * j + 5]),
+                                 pack_bf16(S[8 * j + 6], S[8 * j + 7]));
+            };
+            write_sprime();
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(BAR(B_VCONV + b));
-            return true;
-        };
-        write_sprime();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(B_S_READY));
-        bool ok = nch > 0 ? convert_v(0) : true;
-        for (int n = 0; ok && n < nch; ++n) {
-            const int sl = n & 1;
-            const int64_t t0 = bos + static_cast<int64_t>(n) * C;
-            const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
-            if (!wait_bar(BAR(B_C1_FULL), n & 1, abort_flag)) break;
-            tc_fence_after();
-            if (t == 0) KDA_TRACE_POINT(n, 9);
-            uint32_t r[32];
-            tmem_ld32(tmem + lane_base + COL_C1, r);
-            tmem_wait_ld();
-            if (t < 64) {
-                // pseudo-values D (row t of the chunk) -> fp16 B operand of the state increment
+            if (lane == 0) mbar_arrive(BAR(CB_S_READY));
+            for (int n = 0; n < nch; ++n) {
+                const int sl = n & 1;
+                const int64_t t0 = bos + static_cast<int64_t>(n) * C;
+                const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
+                if (!wait_bar(BAR(CB_C1_FULL), n & 1, abort_flag)) break;
+                tc_fence_after();
+                if (tid == 128) KDA_TRACE_POINT(n, 9);
+                {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tmem + lane_base + COL_C1 + c0, r0);
+                    tmem_ld32(tmem + lane_base + COL_C1 + c0 + 32, r1);
+                    // value side of this row (U for rows < 64, Aqk U below), fp16
+                    const uint32_t uvb = sbase + CH_SLOT + sl * SET_STRIDE + SET_UV + half * 16384;
+                    tmem_wait_ld();
+                    // x = accumulator + value side, computed 8 columns at a time and stored at once
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    st_shared_v4(sbase + OFF_DL + sw64(t, j),
-                                 pack_f16(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1])),
-                                 pack_f16(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3])),
-                                 pack_f16(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5])),
-                                 pack_f16(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7])));
-                fence_proxy_async_smem();
-            } else {
-                const int rr = t - 64;
-                if (rr < L) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((t0 + rr) * H + h) * D + v0);
-                    const float sc = p.scale;
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 u = ld_shared_v4(uvb + sw128(row, j));
+                        const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+                        uint32_t *rr = j < 4 ? r0 + 8 * j : r1 + 8 * (j - 4);
+                        float x[8];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint4 o;
-                        o.x = pack_bf16(sc * __uint_as_float(r[8 * j]), sc * __uint_as_float(r[8 * j + 1]));
-                        o.y = pack_bf16(sc * __uint_as_float(r[8 * j + 2]), sc * __uint_as_float(r[8 * j + 3]));
-                        o.z = pack_bf16(sc * __uint_as_float(r[8 * j + 4]), sc * __uint_as_float(r[8 * j + 5]));
-                        o.w = pack_bf16(sc * __uint_as_float(r[8 * j + 6]), sc * __uint_as_float(r[8 * j + 7]));
-                        dst[j] = o;
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 uf = __half22float2(*reinterpret_cast<const __half2 *>(&uw[e]));
+                            x[2 * e] = __uint_as_float(rr[2 * e]) + uf.x;
+                            x[2 * e + 1] = __uint_as_float(rr[2 * e + 1]) + uf.y;
+                        }
+                        if (row < 64) {
+                            // pseudo-values D -> fp16 B operand of the state increment
+                            st_shared_v4(sbase + CH_DL + half * 8192 + sw128(row, j), pack_f16(x[0], x[1]),
+                                         pack_f16(x[2], x[3]), pack_f16(x[4], x[5]), pack_f16(x[6], x[7]));
+                        } else {
+                            // output row -> staging tile over the value-side rows just consumed
+                            // (same bytes this thread read above); the store warp writes it out
+                            const float sc = p.scale;
+                            st_shared_v4(uvb + sw128(row, j), pack_bf16(sc * x[0], sc * x[1]),
+                                         pack_bf16(sc * x[2], sc * x[3]), pack_bf16(sc * x[4], sc * x[5]),
+                                         pack_bf16(sc * x[6], sc * x[7]));
+                        }
                     }
+                    fence_proxy_async_smem();
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(BAR(B_C1_FREE));
-                if (t < 64) mbar_arrive(BAR(B_D_READY));
-            }
-            if (n + 1 < nch && !convert_v(n + 1)) break;
-            if (!wait_bar(BAR(B_C3_FULL), n & 1, abort_flag)) break;
-            tc_fence_after();
-            if (t == 0) KDA_TRACE_POINT(n, 10);
-            tmem_ld32(tmem + lane_base + COL_C3, r);
-            tmem_wait_ld();
-            const float dec = reinterpret_cast<const float *>(sgen + OFF_DEC + sl * DEC_BYTES)[t];
+                tc_fence_before();
+                __syncwarp();
+                if (tid == 128) KDA_TRACE_POINT(n, 6);
+                if (lane == 0) {
+                    mbar_arrive(BAR(CB_C1_FREE));
+                    mbar_arrive(BAR(row < 64 ? CB_D_READY : CB_O_READY));
+                }
+                if (!wait_bar(BAR(CB_C3_FULL), n & 1, abort_flag)) break;
+                tc_fence_after();
+                if (tid == 128) KDA_TRACE_POINT(n, 10);
+                {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tmem + lane_base + COL_C3 + c0, r0);
+                    tmem_ld32(tmem + lane_base + COL_C3 + c0 + 32, r1);
+                    tmem_wait_ld();
+                    const float dec =
+                        reinterpret_cast<const float *>(sgen + CH_SLOT + sl * SET_STRIDE + SET_DEC)[row];
 #pragma unroll
-            for (int j = 0; j < NV; ++j) S[j] = fmaf(dec, S[j], __uint_as_float(r[j]));
-            if (n + 1 < nch) {
-                write_sprime();
-                fence_proxy_async_smem();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0 && n + 1 < nch) mbar_arrive(BAR(B_S_READY));
-            // hand slot `sl` on to the producer of chunk n + 2 once all four warps are done with it
-            named_bar_sync(1, 128);
-            if (t == 0) KDA_TRACE_POINT(n, 11);
-            if (t == 0 && n + 2 < nch) {
-                const uint32_t prod = static_cast<uint32_t>((n + 2) % NS);
-                if (prod != rank) mbar_expect_tx(BAR(B_SLOT_FULL + sl), SLOT_TX);
-                mbar_arrive_remote(mapa(BAR(B_SLOT_EMPTY + sl), prod));
-            }
-        }
-        // final state slice
-        if (p.hT && !*abort_flag) {
-            const size_t off = state_base + static_cast<size_t>(t) * D + v0;
-            if (p.hT_fp32) {
-                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.hT) + off);
+                    for (int j = 0; j < 32; ++j) S[j] = fmaf(dec, S[j], __uint_as_float(r0[j]));
 #pragma unroll
-                for (int j = 0; j < NV / 4; ++j) dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
-            } else {
-                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.hT) + off);
+                    for (int j = 0; j < 32; ++j) S[32 + j] = fmaf(dec, S[32 + j], __uint_as_float(r1[j]));
+                }
+                if (tid == 128) KDA_TRACE_POINT(n, 8);
+                if (n + 1 < nch) {
+                    write_sprime();
+                    fence_proxy_async_smem();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (n + 1 < nch) mbar_arrive(BAR(CB_S_READY));
+                    mbar_arrive(BAR(CB_SFREE + sl));
+                }
+                if (tid == 128) KDA_TRACE_POINT(n, 11);
+            }
+            // final state
+            if (p.hT && !*abort_flag) {
+                const size_t off = state_base + static_cast<size_t>(row) * D + c0;
+                if (p.hT_fp32) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.hT) + off);
 #pragma unroll
-                for (int j = 0; j < NV / 8; ++j)
-                    dst[j] = make_uint4(pack_bf16(S[8 * j], S[8 * j + 1]), pack_bf16(S[8 * j + 2], S[8 * j + 3]),
-                                        pack_bf16(S[8 * j + 4], S[8 * j + 5]), pack_bf16(S[8 * j + 6], S[8 * j + 7]));
+                    for (int j = 0; j < 16; ++j)
+                        dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+                } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.hT) + off);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        dst[j] = make_uint4(pack_bf16(S[8 * j], S[8 * j + 1]), pack_bf16(S[8 * j + 2], S[8 * j + 3]),
+                                            pack_bf16(S[8 * j + 4], S[8 * j + 5]),
+                                            pack_bf16(S[8 * j + 6], S[8 * j + 7]));
+                }
             }
         }
     } else {
-        // ============================================================ chunk preparation (w8..w11)
-        const int t = tid - 256;               // key channel in the gate pass; TMEM lane in epilogues
-        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t ws = sbase + OFF_STAGE;
-        float *wsf = reinterpret_cast<float *>(sgen + OFF_STAGE);
-        int kk = 0;
-        for (int m = static_cast<int>(rank); m < nch; m += NS, ++kk) {
-            const int sl = m & 1;
-            const uint32_t slot = sbase + sl * SLOT_BYTES;
-            const int64_t t0 = bos + static_cast<int64_t>(m) * C;
-            const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
-            // my slot must have been released by every CTA (chunk m - 2)
-            if (m >= 2) {
-                const int j = static_cast<int>(rank) >= 2 ? kk : kk - 1;
-                if (!wait_bar(BAR(B_SLOT_EMPTY + sl), j & 1, abort_flag)) break;
-            }
-            if (t == 0) KDA_TRACE_POINT(m, 0);
-            if (t < C) beta_s[t] = t < L ? p.beta[(t0 + t) * H + h] : 0.f;
-            if (!wait_bar(BAR(B_STAGE_FULL), kk & 1, abort_flag)) break;
-            named_bar_sync(2, 128);
-            if (t == 0) KDA_TRACE_POINT(m, 1);
-
-            // -------- S1: running log-decay of channel t, decayed factors (T-format tiles)
-            {
-                const int c = t;
-                const float *gcol = reinterpret_cast<const float *>(sgen + OFF_STAGE + STG_G) + c;
-                const uint16_t *qcol = reinterpret_cast<const uint16_t *>(sgen + OFF_STAGE + STG_Q) + c;
-                const uint16_t *kcol = reinterpret_cast<const uint16_t *>(sgen + OFF_STAGE + STG_K) + c;
-                float ga = 0.f, gl = 0.f;
-                for (int r = 0; r < L; ++r) {
-                    gl += gcol[r * D];
-                    if (r == ANCHOR) ga = gl;
+        // ======================================================================= prep CTA
+        const int first = static_cast<int>(rank) - 1;   // chunks first, first + 3, ...
+        if (warp == 0) {
+            // ---- q, k, g staging loads
+            int kk = 0;
+            for (int m = first; m < nch; m += NPREP, ++kk) {
+                const int32_t row = static_cast<int32_t>(bos + static_cast<int64_t>(m) * C);
+                if (kk >= 1 && !wait_bar(BAR(PB_STAGE_FREE), (kk - 1) & 1, abort_flag)) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(BAR(PB_STAGE_FULL), STAGE_TX);
+                    tma_load_3d(sbase + PR_STG + STG_Q, &maps.q, BAR(PB_STAGE_FULL), 0, h, row);
+                    tma_load_3d(sbase + PR_STG + STG_K, &maps.k, BAR(PB_STAGE_FULL), 0, h, row);
+                    tma_load_3d(sbase + PR_STG + STG_G, &maps.g, BAR(PB_STAGE_FULL), 0, h, row);
                 }
-                if (L <= ANCHOR) ga = gl;
-                const float eca = __expf(gl - ga);
-                float G = 0.f;
-#pragma unroll 1
-                for (int rb = 0; rb < 8; ++rb) {
-                    uint32_t ph[4], pq[4], pc[4], pt[4];
+                __syncwarp();
+                if (kk >= 1 && !wait_bar(BAR(PB_VSTAGE_FREE), (kk - 1) & 1, abort_flag)) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(BAR(PB_VSTAGE_FULL), VSTAGE_TX);
+                    tma_load_3d(sbase + PR_STG + STG_V, &maps.v, BAR(PB_VSTAGE_FULL), 0, h, row);
+                    tma_load_3d(sbase + PR_STG + STG_V + 8192, &maps.v, BAR(PB_VSTAGE_FULL), 64, h, row);
+                }
+                __syncwarp();
+            }
+        } else if (warp == 1) {
+            // ---- prep MMA issuer
+            int kk = 0;
+            for (int m = first; m < nch; m += NPREP, ++kk) {
+                if (!wait_bar(BAR(PB_EW_DONE), kk & 1, abort_flag)) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    // [Kh; Qh] Kc^T : A = Kh^T | Qh^T (MN-major, 64-row blocks 16 KB apart), B = Kc^T
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_f16(tmem + COL_P1, smem_desc(sbase + PR_KH + ks * 2048, 16384, 1024, kSwizzle128),
+                                smem_desc(sbase + PR_KC + ks * 2048, 16384, 1024, kSwizzle128), ID_P1, ks > 0);
+                    mma_commit(BAR(PB_P1_DONE));
+                }
+                __syncwarp();
+                if (!wait_bar(BAR(PB_SOLVE_DONE), kk & 1, abort_flag)) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    // W'^T = Kh^T T'^T (bf16)
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(tmem + COL_W, smem_desc(sbase + PR_KH + ks * 32, 16, 1024, kSwizzle128),
+                                smem_desc(sbase + PR_TB + ks * 32, 16, 1024, kSwizzle128), ID_W, ks > 0);
+                    // [T'; Aqk] T' (fp16); rows 64..127 (Aqk T') are used
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(tmem + COL_AV, smem_desc(sbase + PR_AVT + ks * 32, 16, 1024, kSwizzle128),
+                                smem_desc(sbase + PR_AVT + ks * 2048, 16384, 1024, kSwizzle128), ID_AV, ks > 0);
+                    mma_commit(BAR(PB_WAV_DONE));
+                }
+                __syncwarp();
+                if (!wait_bar(BAR(PB_WEPI_DONE), kk & 1, abort_flag)) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    // W'^T Aqk^T (bf16)
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(tmem + COL_Q, smem_desc(sbase + PR_WP + ks * 32, 16, 1024, kSwizzle128),
+                                smem_desc(sbase + PR_AQB + ks * 32, 16, 1024, kSwizzle128), ID_Q, ks > 0);
+                    // [T'; Aqk T'] V = [U; Aqk U]  (fp16, N = 128)
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(tmem + COL_UV, smem_desc(sbase + PR_AVT + ks * 32, 16, 1024, kSwizzle128),
+                                smem_desc(sbase + PR_STG + STG_V + ks * 2048, 8192, 1024, kSwizzle128), ID_UV,
+                                ks > 0);
+                    mma_commit(BAR(PB_Q_DONE));
+                }
+                __syncwarp();
+            }
+        } else if (warp == 3) {
+            // ---- publisher: finished parts of the operand set (smem) -> ring slot (global),
+            // each by bulk stores as soon as the part is final
+            int kk = 0;
+            for (int m = first; m < nch; m += NPREP, ++kk) {
+                const int r = m % NRING;
+                unsigned char *set = ring + static_cast<uint64_t>(r) * SET_STRIDE;
+                // the ring slot must have been pulled by the chain CTA (chunk m - NRING)
+                if (m >= NRING && !wait_bar(BAR(PB_RING_FREE + r), ((m / NRING) - 1) & 1, abort_flag)) break;
+                if (!wait_bar(BAR(PB_OUTA_READY), kk & 1, abort_flag)) break;
+                if (lane == 0) {
+                    bulk_s2g(set + SET_KT, sbase + PR_KC, 16384);
+                    bulk_commit();
+                }
+                __syncwarp();
+                if (!wait_bar(BAR(PB_OUTB_READY), kk & 1, abort_flag)) break;
+                if (lane == 0) {
+                    bulk_s2g(set + SET_W, sbase + PR_KH, 16384);
+                    bulk_commit();
+                    bulk_wait_read0();
+                    mbar_arrive(BAR(PB_OUTAB_FREE));
+                }
+                __syncwarp();
+                if (!wait_bar(BAR(PB_OUTC_READY), kk & 1, abort_flag)) break;
+                if (lane == 0) {
+                    bulk_s2g(set + SET_Q, sbase + PR_AVT, 16384);
+                    bulk_s2g(set + SET_UV, sbase + PR_AKK, 32768);
+                    bulk_s2g(set + SET_DEC, misc + M_DEC + (kk & 1) * 512, 512);
+                    bulk_commit();
+                    bulk_wait_read0();
+                    mbar_arrive(BAR(PB_OUTC_FREE));
+                    bulk_wait0();
+                    fence_proxy_async_global();
+                    mbar_arrive_remote(mapa(sbase + CH_MISC + M_BAR + 8u * (CB_READY + r), 0));
+                    KDA_TRACE_POINT(m, 8);
+                }
+                __syncwarp();
+            }
+        } else if (warp >= 4) {
+            // ---- chunk preparation: 8 warps, 256 threads. Outgoing tiles are assembled in
+            // dead workspace: Kt^T over Kc^T, -W^T over Kh^T, Qt^T over the AV operand, UV over A/T.
+            const int t = tid - 128;
+            const int q4 = warp & 3, half = (warp - 4) >> 2;
+            const int lrow = q4 * 32 + lane;                 // TMEM lane in the epilogues
+            const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+            float *wsf = reinterpret_cast<float *>(sgen);
+            float *beta_s = reinterpret_cast<float *>(miscg + M_BETA);
+            float *ega_s = reinterpret_cast<float *>(miscg + M_EGA);
+            float *gsum = reinterpret_cast<float *>(miscg + M_GSUM);
+            float *dec_all = reinterpret_cast<float *>(miscg + M_DEC);
+            int kk = 0;
+            for (int m = first; m < nch; m += NPREP, ++kk) {
+                const int64_t t0 = bos + static_cast<int64_t>(m) * C;
+                const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
+                if (*abort_flag) break;
+                if (t == 0) KDA_TRACE_POINT(m, 0);
+                if (t < C) beta_s[t] = t < L ? p.beta[(t0 + t) * H + h] : 0.f;
+                // parts A and B of the previous set must have been read out by the publisher
+                if (kk >= 1 && !wait_bar(BAR(PB_OUTAB_FREE), (kk - 1) & 1, abort_flag)) break;
+                if (!wait_bar(BAR(PB_STAGE_FULL), kk & 1, abort_flag)) break;
+                if (t == 0) KDA_TRACE_POINT(m, 1);
+
+                // -------- S1: running log-decay, two threads per channel (rows 0-31 / 32-63)
+                uint32_t ktr[16];   // Kt^T row of this thread (fp16 pairs), stored after the S2 MMA
+                {
+                    const int c = t & 127, hr = t >> 7;
+                    const float *gcol = reinterpret_cast<const float *>(sgen + PR_STG + STG_G) + c;
+                    const uint16_t *qcol = reinterpret_cast<const uint16_t *>(sgen + PR_STG + STG_Q) + c;
+                    const uint16_t *kcol = reinterpret_cast<const uint16_t *>(sgen + PR_STG + STG_K) + c;
+                    float gv[32];
+                    float part = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float kh[2], qh[2], kc[2], kt[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int r = rb * 8 + 2 * e + u;
-                            const bool valid = r < L;
-                            G += valid ? gcol[r * D] : 0.f;
-                            const float x = G - ga;
-                            const float ep = __expf(x), em = __expf(-x);
-                            const float kv = valid ? bf2f(kcol[r * D]) : 0.f;
-                            const float qv = valid ? bf2f(qcol[r * D]) : 0.f;
-                            kh[u] = kv * ep;
-                            qh[u] = qv * ep;
-                            kc[u] = kv * em;
-                            kt[u] = kc[u] * eca;
-                        }
-                        ph[e] = pack_bf16(kh[0], kh[1]);
-                        pq[e] = pack_bf16(qh[0], qh[1]);
-                        pc[e] = pack_bf16(kc[0], kc[1]);
-                        pt[e] = pack_f16(kt[0], kt[1]);
+                    for (int i = 0; i < 32; ++i) {
+                        const int rr = hr * 32 + i;
+                        gv[i] = rr < L ? gcol[rr * D] : 0.f;
+                        part += gv[i];
                     }
-                    const uint32_t o = sw128(c, rb);
-                    st_shared_v4(slot + SLOT_W + o, ph[0], ph[1], ph[2], ph[3]);   // Kh^T (scratch)
-                    st_shared_v4(slot + SLOT_Q + o, pq[0], pq[1], pq[2], pq[3]);   // Qh^T (scratch)
-                    st_shared_v4(slot + SLOT_AV + o, pc[0], pc[1], pc[2], pc[3]);  // Kc^T (scratch)
-                    st_shared_v4(slot + SLOT_KT + o, pt[0], pt[1], pt[2], pt[3]);  // Kt^T
-                }
-                reinterpret_cast<float *>(sgen + OFF_DEC + sl * DEC_BYTES)[c] = __expf(gl);
-                ega_s[c] = __expf(ga);
-            }
-            fence_proxy_async_smem();
-            named_bar_sync(2, 128);
-            if (t == 0) { mbar_arrive(BAR(B_EW_DONE)); KDA_TRACE_POINT(m, 2); }
-
-            // -------- S2 epilogue: A (fp32, masked, beta-scaled) and Aqk (fp16 + bf16)
-            if (!wait_bar(BAR(B_P1_DONE), kk & 1, abort_flag)) break;
-            tc_fence_after();
-            if (t == 0) KDA_TRACE_POINT(m, 3);
-            {
-                uint32_t a0[32], a1[32];
-                tmem_ld32(tmem + lane_base + COL_P1, a0);
-                tmem_ld32(tmem + lane_base + COL_P1 + 32, a1);
-                tmem_wait_ld();
-                if (t < 64) {
-                    const int r = t;
-                    const float br = beta_s[r];
-                    float *row = wsf + WS_AKK / 4 + r * AKK_LD;
+                    gsum[hr * 128 + c] = part;
+                    named_bar_sync(2, 256);
+                    const float ga = gsum[c];                   // G at the anchor row 31
+                    const float gl = ga + gsum[128 + c];        // G at the last row
+                    const float eca = __expf(gl - ga);
+                    float G = hr ? ga : 0.f;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        float v4[4];
+                    for (int rb = 0; rb < 4; ++rb) {
+                        uint32_t ph[4], pq[4], pc[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int i = 4 * j + e;
-                            const float a = __uint_as_float(i < 32 ? a0[i] : a1[i - 32]);
-                            v4[e] = i < r ? br * a : 0.f;
+                            float kh[2], qh[2], kc[2], kt[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const int i = rb * 8 + 2 * e + u, rr = hr * 32 + i;
+                                const bool valid = rr < L;
+                                G += gv[i];
+                                const float x = G - ga;
+                                const float ep = __expf(x), em = __expf(-x);
+                                const float kv = valid ? bf2f(kcol[rr * D]) : 0.f;
+                                const float qv = valid ? bf2f(qcol[rr * D]) : 0.f;
+                                kh[u] = kv * ep;
+                                qh[u] = qv * ep;
+                                kc[u] = kv * em;
+                                kt[u] = kc[u] * eca;
+                            }
+                            ph[e] = pack_bf16(kh[0], kh[1]);
+                            pq[e] = pack_bf16(qh[0], qh[1]);
+                            pc[e] = pack_bf16(kc[0], kc[1]);
+                            ktr[rb * 4 + e] = pack_f16(kt[0], kt[1]);
                         }
-                        *reinterpret_cast<float4 *>(row + 4 * j) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+                        const uint32_t o = sw128(c, hr * 4 + rb);
+                        st_shared_v4(sbase + PR_KH + o, ph[0], ph[1], ph[2], ph[3]);
+                        st_shared_v4(sbase + PR_QH + o, pq[0], pq[1], pq[2], pq[3]);
+                        st_shared_v4(sbase + PR_KC + o, pc[0], pc[1], pc[2], pc[3]);
                     }
-                } else {
-                    const int r = t - 64;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        float v8[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int i = 8 * j + e;
-                            const float a = __uint_as_float(i < 32 ? a0[i] : a1[i - 32]);
-                            v8[e] = i <= r ? a : 0.f;
-                        }
-                        st_shared_v4(slot + SLOT_AV + sw128(64 + r, j), pack_f16(v8[0], v8[1]),
-                                     pack_f16(v8[2], v8[3]), pack_f16(v8[4], v8[5]), pack_f16(v8[6], v8[7]));
-                        st_shared_v4(ws + WS_AQB + sw128(r, j), pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]),
-                                     pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
+                    if (hr == 0) {
+                        dec_all[(kk & 1) * 128 + c] = __expf(gl);
+                        ega_s[c] = __expf(ga);
                     }
                 }
-            }
-            tc_fence_before();
-            named_bar_sync(2, 128);
+                fence_proxy_async_smem();
+                named_bar_sync(2, 256);
+                if (t == 0) {
+                    mbar_arrive(BAR(PB_EW_DONE));
+                    mbar_arrive(BAR(PB_STAGE_FREE));
+                    KDA_TRACE_POINT(m, 2);
+                }
+                // value tile bf16 -> fp16 in place (B operand of the value-side MMA)
+                if (!wait_bar(BAR(PB_VSTAGE_FULL), kk & 1, abort_flag)) break;
+#pragma unroll
+                for (int c2 = 0; c2 < 4; ++c2) {
+                    const uint32_t a = sbase + PR_STG + STG_V + (t + 256 * c2) * 16;
+                    const uint4 x = ld_shared_v4(a);
+                    st_shared_v4(a, pack_f16(lo_bf(x.x), hi_bf(x.x)), pack_f16(lo_bf(x.y), hi_bf(x.y)),
+                                 pack_f16(lo_bf(x.z), hi_bf(x.z)), pack_f16(lo_bf(x.w), hi_bf(x.w)));
+                }
+                fence_proxy_async_smem();
 
-            // -------- S3: T = (I + A)^-1, blocked forward substitution on 16 x 16 blocks
-            {
-                const float *A = wsf + WS_AKK / 4;
-                float *T = wsf + WS_T / 4;
-                float *P = wsf + WS_P / 4;
-                // diagonal blocks: warp w inverts block w, lane i < 16 owns column i
-                const int wb = t >> 5, li = t & 31;
-                if (li < 16) {
-                    float x[16];
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        float acc = (r == li) ? 1.f : 0.f;
-                        const float *arow = A + (16 * wb + r) * AKK_LD + 16 * wb;
-#pragma unroll
-                        for (int j = 0; j < r; ++j) acc = fmaf(-arow[j], x[j], acc);
-                        x[r] = acc;
-                    }
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) T[(16 * wb + r) * AKK_LD + 16 * wb + li] = x[r];
-                }
-                named_bar_sync(2, 128);
-                // off-diagonal blocks by distance d = I - J: T_IJ = -T_II * sum_{K=J}^{I-1} A_IK T_KJ
-#pragma unroll 1
-                for (int d = 1; d < 4; ++d) {
-                    const int nb = 4 - d;
-                    for (int e = t; e < nb * 256; e += 128) {
-                        const int J = e >> 8, I = J + d, r = (e >> 4) & 15, c = e & 15;
-                        float acc = 0.f;
-                        for (int K = J; K < I; ++K) {
-                            const float *arow = A + (16 * I + r) * AKK_LD + 16 * K;
-                            const float *tcol = T + (16 * K) * AKK_LD + 16 * J + c;
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) acc = fmaf(arow[j], tcol[j * AKK_LD], acc);
-                        }
-                        P[J * 256 + r * 16 + c] = acc;
-                    }
-                    named_bar_sync(2, 128);
-                    for (int e = t; e < nb * 256; e += 128) {
-                        const int J = e >> 8, I = J + d, r = (e >> 4) & 15, c = e & 15;
-                        const float *trow = T + (16 * I + r) * AKK_LD + 16 * I;
-                        float acc = 0.f;
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) acc = fmaf(trow[j], P[J * 256 + j * 16 + c], acc);
-                        T[(16 * I + r) * AKK_LD + 16 * J + c] = -acc;
-                    }
-                    named_bar_sync(2, 128);
-                }
-                // T' = T diag(beta): fp16 into the slot's AV rows 0..63, bf16 into the workspace
+                // -------- S2 epilogue: A (fp32, masked, beta-scaled) and Aqk (fp16 + bf16); Kt^T out
+                // (part C of the previous set, over A / T and the AV operand, must be read out)
+                if (kk >= 1 && !wait_bar(BAR(PB_OUTC_FREE), (kk - 1) & 1, abort_flag)) break;
+                if (!wait_bar(BAR(PB_P1_DONE), kk & 1, abort_flag)) break;
+                tc_fence_after();
+                if (t == 0) KDA_TRACE_POINT(m, 3);
                 {
-                    const int r = t >> 1, half = t & 1;
+                    const int c = t & 127, hr = t >> 7;
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const int j = half * 4 + jj;
-                        float v8[8];
+                    for (int rb = 0; rb < 4; ++rb)
+                        st_shared_v4(sbase + PR_KC + sw128(c, hr * 4 + rb), ktr[rb * 4], ktr[rb * 4 + 1],
+                                     ktr[rb * 4 + 2], ktr[rb * 4 + 3]);
+                    uint32_t a[32];
+                    tmem_ld32(tmem + lane_base + COL_P1 + half * 32, a);
+                    tmem_wait_ld();
+                    if (lrow < 64) {
+                        const int rr = lrow;
+                        const float br = beta_s[rr];
+                        float *rowp = wsf + PR_AKK / 4 + rr * AKK_LD + half * 32;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int i = 8 * j + e;
-                            v8[e] = i <= r ? T[r * AKK_LD + i] * beta_s[i] : 0.f;
+                        for (int j = 0; j < 8; ++j) {
+                            float v4[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int i = half * 32 + 4 * j + e;
+                                v4[e] = i < rr ? br * __uint_as_float(a[4 * j + e]) : 0.f;
+                            }
+                            *reinterpret_cast<float4 *>(rowp + 4 * j) = make_float4(v4[0], v4[1], v4[2], v4[3]);
                         }
-                        st_shared_v4(slot + SLOT_AV + sw128(r, j), pack_f16(v8[0], v8[1]), pack_f16(v8[2], v8[3]),
-                                     pack_f16(v8[4], v8[5]), pack_f16(v8[6], v8[7]));
-                        // WS_TB overlays the fp32 A block; A is no longer read after the barrier above
-                        st_shared_v4(ws + WS_TB + sw128(r, j), pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]),
-                                     pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
+                    } else {
+                        const int rr = lrow - 64;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            float v8[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int i = half * 32 + 8 * j + e;
+                                v8[e] = i <= rr ? __uint_as_float(a[8 * j + e]) : 0.f;
+                            }
+                            const int jj = half * 4 + j;
+                            st_shared_v4(sbase + PR_AVT + sw128(64 + rr, jj), pack_f16(v8[0], v8[1]),
+                                         pack_f16(v8[2], v8[3]), pack_f16(v8[4], v8[5]), pack_f16(v8[6], v8[7]));
+                            st_shared_v4(sbase + PR_AQB + sw128(rr, jj), pack_bf16(v8[0], v8[1]),
+                                         pack_bf16(v8[2], v8[3]), pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
+                        }
+                    }
+                    // blocks of T read as zeros by the fixed-length products below
+                    float *T = wsf + PR_T / 4;
+                    T[(t >> 4) * AKK_LD + 16 + (t & 15)] = 0.f;               // rows 0-15, cols 16-31
+                    T[(32 + (t >> 4)) * AKK_LD + 48 + (t & 15)] = 0.f;        // rows 32-47, cols 48-63
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(2, 256);
+                if (t == 0) {
+                    mbar_arrive(BAR(PB_OUTA_READY));
+                    KDA_TRACE_POINT(m, 9);
+                }
+
+                // -------- S3: T = (I + A)^-1 by recursive blocking:
+                //   (a) the four 16 x 16 diagonal blocks by forward substitution,
+                //   (b) the two 16 x 16 blocks below them inside each 32 x 32 diagonal block,
+                //   (c) the 32 x 32 block below the diagonal,
+                // each off-diagonal block as  T_IJ = -T_II (A_IJ T_JJ).
+                {
+                    const float *A = wsf + PR_AKK / 4;
+                    float *T = wsf + PR_T / 4;
+                    float *P = wsf + PR_P / 4;
+                    if (t < 128) {
+                        const int wb = t >> 5, li = t & 31;
+                        if (li < 16) {
+                            float x[16];
+#pragma unroll
+                            for (int rr = 0; rr < 16; ++rr) {
+                                const float *arow = A + (16 * wb + rr) * AKK_LD + 16 * wb;
+                                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                                for (int j = 0; j < rr; ++j) {
+                                    const float pr = arow[j] * x[j];
+                                    if ((j & 3) == 0) a0 += pr;
+                                    else if ((j & 3) == 1) a1 += pr;
+                                    else if ((j & 3) == 2) a2 += pr;
+                                    else a3 += pr;
+                                }
+                                x[rr] = ((rr == li) ? 1.f : 0.f) - ((a0 + a1) + (a2 + a3));
+                            }
+#pragma unroll
+                            for (int rr = 0; rr < 16; ++rr) T[(16 * wb + rr) * AKK_LD + 16 * wb + li] = x[rr];
+                        }
+                    }
+                    named_bar_sync(2, 256);
+                    if (t == 0) KDA_TRACE_POINT(m, 10);
+                    // (b) blocks (1,0) and (3,2): P = A_IJ T_JJ, then T_IJ = -T_II P (two columns per thread)
+                    {
+                        const int blk = t >> 7, rr = (t >> 3) & 15, cc = (t & 7) * 2;
+                        const int J = 2 * blk, I = J + 1;
+                        const float *arow = A + (16 * I + rr) * AKK_LD + 16 * J;
+                        float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float a = arow[j];
+                            const float2 tv = *reinterpret_cast<const float2 *>(T + (16 * J + j) * AKK_LD + 16 * J + cc);
+                            p0 = fmaf(a, tv.x, p0);
+                            p1 = fmaf(a, tv.y, p1);
+                        }
+                        *reinterpret_cast<float2 *>(P + blk * 256 + rr * 16 + cc) = make_float2(p0, p1);
+                        named_bar_sync(2, 256);
+                        const float *trow = T + (16 * I + rr) * AKK_LD + 16 * I;
+                        p0 = 0.f;
+                        p1 = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float a = trow[j];
+                            const float2 pv = *reinterpret_cast<const float2 *>(P + blk * 256 + j * 16 + cc);
+                            p0 = fmaf(a, pv.x, p0);
+                            p1 = fmaf(a, pv.y, p1);
+                        }
+                        *reinterpret_cast<float2 *>(T + (16 * I + rr) * AKK_LD + 16 * J + cc) = make_float2(-p0, -p1);
+                    }
+                    named_bar_sync(2, 256);
+                    if (t == 0) KDA_TRACE_POINT(m, 11);
+                    // (c) rows 32..63, columns 0..31: P2 = A[32:, :32] T[:32, :32]; T = -T[32:, 32:] P2
+                    {
+                        const int rr = t >> 3, c4 = (t & 7) * 4;
+                        const float *arow = A + (32 + rr) * AKK_LD;
+                        float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float a = arow[j];
+                            const float4 tv = *reinterpret_cast<const float4 *>(T + j * AKK_LD + c4);
+                            p0 = fmaf(a, tv.x, p0);
+                            p1 = fmaf(a, tv.y, p1);
+                            p2 = fmaf(a, tv.z, p2);
+                            p3 = fmaf(a, tv.w, p3);
+                        }
+                        *reinterpret_cast<float4 *>(P + rr * 32 + c4) = make_float4(p0, p1, p2, p3);
+                        named_bar_sync(2, 256);
+                        const float *trow = T + (32 + rr) * AKK_LD + 32;
+                        p0 = p1 = p2 = p3 = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float a = trow[j];
+                            const float4 pv = *reinterpret_cast<const float4 *>(P + j * 32 + c4);
+                            p0 = fmaf(a, pv.x, p0);
+                            p1 = fmaf(a, pv.y, p1);
+                            p2 = fmaf(a, pv.z, p2);
+                            p3 = fmaf(a, pv.w, p3);
+                        }
+                        *reinterpret_cast<float4 *>(T + (32 + rr) * AKK_LD + c4) = make_float4(-p0, -p1, -p2, -p3);
+                    }
+                    named_bar_sync(2, 256);
+                    if (t == 0) KDA_TRACE_POINT(m, 12);
+                    // T' = T diag(beta): fp16 -> AV rows 0..63, bf16 -> TB
+                    {
+                        const int rr = t >> 2, qt = t & 3;
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const int j = qt * 2 + jj;
+                            const float4 ta = *reinterpret_cast<const float4 *>(T + rr * AKK_LD + 8 * j);
+                            const float4 tb = *reinterpret_cast<const float4 *>(T + rr * AKK_LD + 8 * j + 4);
+                            const float4 ba = *reinterpret_cast<const float4 *>(beta_s + 8 * j);
+                            const float4 bb = *reinterpret_cast<const float4 *>(beta_s + 8 * j + 4);
+                            const float tvv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+                            const float bvv[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+                            float v8[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) v8[e] = (8 * j + e) <= rr ? tvv[e] * bvv[e] : 0.f;
+                            st_shared_v4(sbase + PR_AVT + sw128(rr, j), pack_f16(v8[0], v8[1]), pack_f16(v8[2], v8[3]),
+                                         pack_f16(v8[4], v8[5]), pack_f16(v8[6], v8[7]));
+                            st_shared_v4(sbase + PR_TB + sw128(rr, j), pack_bf16(v8[0], v8[1]),
+                                         pack_bf16(v8[2], v8[3]), pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
+                        }
                     }
                 }
-            }
-            fence_proxy_async_smem();
-            named_bar_sync(2, 128);
-            if (t == 0) { mbar_arrive(BAR(B_SOLVE_DONE)); KDA_TRACE_POINT(m, 4); }
-
-            // -------- S4 epilogues: W (anchored copy + final negated/unanchored), Aqk T'
-            if (!wait_bar(BAR(B_WAV_DONE), kk & 1, abort_flag)) break;
-            tc_fence_after();
-            if (t == 0) KDA_TRACE_POINT(m, 5);
-            {
-                uint32_t a0[32], a1[32];
-                tmem_ld32(tmem + lane_base + COL_W, a0);
-                tmem_ld32(tmem + lane_base + COL_W + 32, a1);
-                tmem_wait_ld();
-                const float sc = -ega_s[t];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    float v8[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v8[e] = __uint_as_float(j < 4 ? a0[8 * j + e] : a1[8 * (j - 4) + e]);
-                    st_shared_v4(ws + WS_WP + sw128(t, j), pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]),
-                                 pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
-                    st_shared_v4(slot + SLOT_W + sw128(t, j), pack_bf16(sc * v8[0], sc * v8[1]),
-                                 pack_bf16(sc * v8[2], sc * v8[3]), pack_bf16(sc * v8[4], sc * v8[5]),
-                                 pack_bf16(sc * v8[6], sc * v8[7]));
+                fence_proxy_async_smem();
+                named_bar_sync(2, 256);
+                if (t == 0) {
+                    mbar_arrive(BAR(PB_SOLVE_DONE));
+                    KDA_TRACE_POINT(m, 4);
                 }
-                if (t >= 64) {
-                    tmem_ld32(tmem + lane_base + COL_AV, a0);
-                    tmem_ld32(tmem + lane_base + COL_AV + 32, a1);
+
+                // -------- S4 epilogues: W (anchored copy; final -W unanchored over Kh^T), Aqk T'
+                if (!wait_bar(BAR(PB_WAV_DONE), kk & 1, abort_flag)) break;
+                tc_fence_after();
+                if (t == 0) KDA_TRACE_POINT(m, 5);
+                {
+                    uint32_t a[32];
+                    tmem_ld32(tmem + lane_base + COL_W + half * 32, a);
                     tmem_wait_ld();
+                    const float sc = -ega_s[lrow];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float v8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v8[e] = __uint_as_float(a[8 * j + e]);
+                        const int jj = half * 4 + j;
+                        st_shared_v4(sbase + PR_WP + sw128(lrow, jj), pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]),
+                                     pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
+                        st_shared_v4(sbase + PR_KH + sw128(lrow, jj), pack_bf16(sc * v8[0], sc * v8[1]),
+                                     pack_bf16(sc * v8[2], sc * v8[3]), pack_bf16(sc * v8[4], sc * v8[5]),
+                                     pack_bf16(sc * v8[6], sc * v8[7]));
+                    }
+                    if (lrow >= 64) {
+                        // Aqk T' -> rows 64..127 of the value-side A operand
+                        tmem_ld32(tmem + lane_base + COL_AV + half * 32, a);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int jj = half * 4 + j;
+                            st_shared_v4(sbase + PR_AVT + sw128(lrow, jj),
+                                         pack_f16(__uint_as_float(a[8 * j]), __uint_as_float(a[8 * j + 1])),
+                                         pack_f16(__uint_as_float(a[8 * j + 2]), __uint_as_float(a[8 * j + 3])),
+                                         pack_f16(__uint_as_float(a[8 * j + 4]), __uint_as_float(a[8 * j + 5])),
+                                         pack_f16(__uint_as_float(a[8 * j + 6]), __uint_as_float(a[8 * j + 7])));
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(2, 256);
+                if (t == 0) {
+                    mbar_arrive(BAR(PB_WEPI_DONE));
+                    mbar_arrive(BAR(PB_OUTB_READY));
+                    KDA_TRACE_POINT(m, 6);
+                }
+
+                // -------- Qt = (Qh - Aqk W') e^Ga (over the AV operand) and UV (over A / T)
+                if (!wait_bar(BAR(PB_Q_DONE), kk & 1, abort_flag)) break;
+                tc_fence_after();
+                if (t == 0) KDA_TRACE_POINT(m, 7);
+                {
+                    uint32_t a[32];
+                    tmem_ld32(tmem + lane_base + COL_Q + half * 32, a);
+                    tmem_wait_ld();
+                    const float sc = ega_s[lrow];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int jj = half * 4 + j;
+                        const uint4 qv = ld_shared_v4(sbase + PR_QH + sw128(lrow, jj));
+                        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            o[e] = pack_bf16(sc * (lo_bf(qw[e]) - __uint_as_float(a[8 * j + 2 * e])),
+                                             sc * (hi_bf(qw[e]) - __uint_as_float(a[8 * j + 2 * e + 1])));
+                        st_shared_v4(sbase + PR_AVT + sw128(lrow, jj), o[0], o[1], o[2], o[3]);
+                    }
+                    if (t == 0) KDA_TRACE_POINT(m, 14);
+                    // value side UV = [U; Aqk U], row lrow, 64 columns of block `half`
+                    uint32_t u0[32], u1[32];
+                    tmem_ld32(tmem + lane_base + COL_UV + half * 64, u0);
+                    tmem_ld32(tmem + lane_base + COL_UV + half * 64 + 32, u1);
+                    tmem_wait_ld();
+                    const uint32_t uvb = sbase + PR_AKK + half * 16384;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        float v8[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            v8[e] = __uint_as_float(j < 4 ? a0[8 * j + e] : a1[8 * (j - 4) + e]);
-                        st_shared_v4(slot + SLOT_AV + sw128(t, j), pack_f16(v8[0], v8[1]), pack_f16(v8[2], v8[3]),
-                                     pack_f16(v8[4], v8[5]), pack_f16(v8[6], v8[7]));
+                        const uint32_t *x = j < 4 ? u0 + 8 * j : u1 + 8 * (j - 4);
+                        st_shared_v4(uvb + sw128(lrow, j), pack_f16(__uint_as_float(x[0]), __uint_as_float(x[1])),
+                                     pack_f16(__uint_as_float(x[2]), __uint_as_float(x[3])),
+                                     pack_f16(__uint_as_float(x[4]), __uint_as_float(x[5])),
+                                     pack_f16(__uint_as_float(x[6]), __uint_as_float(x[7])));
                     }
                 }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar_sync(2, 128);
-            if (t == 0) { mbar_arrive(BAR(B_WEPI_DONE)); KDA_TRACE_POINT(m, 6); }
-
-            // -------- Qt = (Qh - Aqk W') e^Ga, row t of Qt^T, in place over Qh^T
-            if (!wait_bar(BAR(B_Q_DONE), kk & 1, abort_flag)) break;
-            tc_fence_after();
-            if (t == 0) KDA_TRACE_POINT(m, 7);
-            {
-                uint32_t a0[32], a1[32];
-                tmem_ld32(tmem + lane_base + COL_Q, a0);
-                tmem_ld32(tmem + lane_base + COL_Q + 32, a1);
-                tmem_wait_ld();
-                const float sc = ega_s[t];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 qv = ld_shared_v4(slot + SLOT_Q + sw128(t, j));
-                    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-                    uint32_t o[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float c0 = __uint_as_float(j < 4 ? a0[8 * j + 2 * e] : a1[8 * (j - 4) + 2 * e]);
-                        const float c1 = __uint_as_float(j < 4 ? a0[8 * j + 2 * e + 1] : a1[8 * (j - 4) + 2 * e + 1]);
-                        const float q0 = __uint_as_float(qw[e] << 16), q1 = __uint_as_float(qw[e] & 0xFFFF0000u);
-                        o[e] = pack_bf16(sc * (q0 - c0), sc * (q1 - c1));
-                    }
-                    st_shared_v4(slot + SLOT_Q + sw128(t, j), o[0], o[1], o[2], o[3]);
+                if (t == 0) KDA_TRACE_POINT(m, 15);
+                // hand the finished set to the publisher
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(2, 256);
+                if (t == 0) {
+                    mbar_arrive(BAR(PB_VSTAGE_FREE));
+                    mbar_arrive(BAR(PB_OUTC_READY));
                 }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar_sync(2, 128);
-            if (t == 0) {
-                mbar_arrive(BAR(B_STAGE_FREE));
-                // publish the slot: bulk copies to the three peers, then one arrival each
-                const uint32_t full = BAR(B_SLOT_FULL + sl);
-                for (uint32_t pr = 0; pr < NS; ++pr) {
-                    if (pr == rank) continue;
-                    const uint32_t rfull = mapa(full, pr);
-                    for (uint32_t part = 0; part < 4; ++part)
-                        bulk_copy_to_peer(mapa(slot + part * 16384, pr), slot + part * 16384, 16384, rfull);
-                    bulk_copy_to_peer(mapa(sbase + OFF_DEC + sl * DEC_BYTES, pr), sbase + OFF_DEC + sl * DEC_BYTES,
-                                      DEC_BYTES, rfull);
-                    mbar_arrive_remote(rfull);
-                }
-                mbar_arrive(full);
-                KDA_TRACE_POINT(m, 8);
             }
         }
     }
@@ -820,6 +1067,22 @@ bool encode3d(CUtensorMap *map, const void *base, CUtensorMapDataType dt, uint32
     return r == CUDA_SUCCESS;
 }
 
+// Per-device ring pool of the operand-set exchange, allocated on first use and
+// held for the life of the process.
+std::mutex g_pool_mu;
+unsigned char *g_pool[64] = {};
+
+unsigned char *ring_pool(int dev) {
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(g_pool_mu);
+    if (!g_pool[dev]) {
+        void *ptr = nullptr;
+        if (cudaMalloc(&ptr, static_cast<size_t>(tc::kMaxRings) * tc::RING_BYTES) != cudaSuccess) return nullptr;
+        g_pool[dev] = static_cast<unsigned char *>(ptr);
+    }
+    return g_pool[dev];
+}
+
 }  // namespace
 
 cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream) {
@@ -827,6 +1090,11 @@ cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream)
     if (units == 0) return cudaSuccess;
     const int64_t grid = units * tc::NS;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    unsigned char *rings = ring_pool(dev);
+    if (!rings) return cudaErrorMemoryAllocation;
     tc::TmaMaps maps;
     memset(&maps, 0, sizeof(maps));
     if (rows > 0) {
@@ -837,12 +1105,14 @@ cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream)
                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
             !encode3d(&maps.g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.num_heads, rows, 128,
                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
-            !encode3d(&maps.v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.num_heads, rows, tc::NV,
-                      CU_TENSOR_MAP_SWIZZLE_64B))
+            !encode3d(&maps.v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.num_heads, rows, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode3d(&maps.o, p.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.num_heads, rows, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
-    cudaError_t err = cudaFuncSetAttribute(tc::kda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(tc::SMEM_BYTES));
+    err = cudaFuncSetAttribute(tc::kda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(tc::SMEM_BYTES));
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -856,7 +1126,7 @@ cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, tc::kda_fwd_tc_kernel, p, maps);
+    err = cudaLaunchKernelEx(&cfg, tc::kda_fwd_tc_kernel, p, maps, rings);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
