@@ -24,7 +24,10 @@
  *  - Argument errors are detected before anything is enqueued and returned as
  *    a kda_status; nothing is written then. Launch failures return
  *    KDA_ERR_CUDA (the CUDA error is left for cudaGetLastError()).
- *  - The library allocates no device memory in kda_fwd.
+ *  - kda_fwd allocates, on its first call on each device, one 123 MiB scratch
+ *    pool (the operand-set rings of its kernel, 256 x 492 KiB) and holds it for
+ *    the life of the process; later calls allocate nothing. kda_fwd_noalloc
+ *    never allocates (see there).
  */
 #ifndef KDA_H_
 #define KDA_H_
@@ -47,7 +50,8 @@ typedef enum {
     KDA_ERR_UNSUPPORTED_DEVICE = 6,/* the current device is not sm_100 (B200 class)      */
     KDA_ERR_BAD_ALIGNMENT = 7,     /* a tensor pointer is not 16-byte aligned            */
     KDA_ERR_TOO_LARGE = 8,         /* sizes exceed what the library indexes              */
-    KDA_ERR_TIMEOUT = 9            /* a kernel gave up on a bounded wait (see kda_device_error) */
+    KDA_ERR_TIMEOUT = 9,           /* a kernel gave up on a bounded wait (see kda_device_error) */
+    KDA_ERR_NOALLOC_LIMIT = 10     /* kda_fwd_noalloc: more (sequence, head) pairs than its scratch holds */
 } kda_status;
 
 typedef enum { KDA_DTYPE_NONE = 0, KDA_DTYPE_BF16 = 1, KDA_DTYPE_FP32 = 2 } kda_dtype;
@@ -97,6 +101,42 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
                    int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
                    kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype,
                    void *out, kda_stream_t stream);
+
+/*
+ * kda_fwd_noalloc -- kda_fwd for callers that cannot allocate device memory.
+ *
+ * The method's pages define no such call; it exists for the library's own
+ * callers. Some cannot let a library allocate: a process whose device memory is
+ * handed out entirely by its own pool or by a framework's caching allocator, a
+ * caller that must keep its memory footprint fixed once it has started serving,
+ * or code that enqueues work where an allocation would stall or be refused.
+ * kda_fwd's scratch pool is allocated on its first call on a device; this entry
+ * point uses instead a scratch array that is part of the library's device image
+ * (KDA_NOALLOC_MAX_UNITS operand-set rings, 15.4 MiB, present once the library's
+ * kernels are loaded on the device), and calls no allocating routine at all.
+ *
+ * Arguments, layouts, results and status codes are those of kda_fwd, plus:
+ *  - num_seqs_eff * num_heads must not exceed KDA_NOALLOC_MAX_UNITS (32): one
+ *    ring of the scratch per (sequence, head) pair. A larger call returns
+ *    KDA_ERR_NOALLOC_LIMIT before anything is enqueued; split it, or use kda_fwd.
+ *  - The first call on each device looks up the scratch's device address (the
+ *    device must be current; a failed lookup returns KDA_ERR_CUDA) and may load
+ *    the library's kernels onto the device. Make that first call before any
+ *    stream capture begins.
+ *  - The scratch is shared by every call on a device: two kda_fwd_noalloc calls
+ *    whose work overlaps in time (on different streams, or from different host
+ *    threads without ordering) race on it and give wrong results. Order them on
+ *    one stream, or use kda_fwd, whose kernels never share a ring.
+ *  - Nothing in the scratch needs to start at zero, and the call clears nothing:
+ *    every ring slot is written by the kernel before the kernel reads it.
+ */
+#define KDA_NOALLOC_MAX_UNITS 32
+kda_status kda_fwd_noalloc(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, float scale, const int32_t *cu_seqlens,
+                           int32_t num_seqs, int32_t batch, int64_t seq_len, int32_t num_heads,
+                           int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
+                           kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype,
+                           void *out, kda_stream_t stream);
 
 /*
  * kda_device_error -- synchronise the current device, then read and clear the

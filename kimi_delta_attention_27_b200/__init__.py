@@ -16,7 +16,10 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libkda.so")
 
 # entry points declared in include/kda.h
-EXPORTS = ("kda_device_error", "kda_fwd", "kda_status_string", "kda_version")
+EXPORTS = ("kda_device_error", "kda_fwd", "kda_fwd_noalloc", "kda_status_string", "kda_version")
+
+# (sequence, head) pairs per kda_fwd_noalloc call (KDA_NOALLOC_MAX_UNITS in include/kda.h)
+NOALLOC_MAX_UNITS = 32
 
 KDA_DTYPE_NONE, KDA_DTYPE_BF16, KDA_DTYPE_FP32 = 0, 1, 2
 
@@ -44,9 +47,11 @@ def load_library(path: str | None = None):
                                "(run python -m kimi_delta_attention_27_b200.build)")
         lib = ctypes.CDLL(p)
         P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
-        lib.kda_fwd.restype = ctypes.c_int
-        lib.kda_fwd.argtypes = [P, P, P, P, P, ctypes.c_float, P, i32, i32, i64, i32, i32, i32,
-                                P, ctypes.c_int, P, ctypes.c_int, P, P]
+        fwd_args = [P, P, P, P, P, ctypes.c_float, P, i32, i32, i64, i32, i32, i32,
+                    P, ctypes.c_int, P, ctypes.c_int, P, P]
+        for name in ("kda_fwd", "kda_fwd_noalloc"):
+            getattr(lib, name).restype = ctypes.c_int
+            getattr(lib, name).argtypes = fwd_args
         lib.kda_status_string.restype = ctypes.c_char_p
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_version.restype = ctypes.c_int32
@@ -108,6 +113,28 @@ def kda_fwd(q, k, v, g, beta, scale: float | None = None, cu_seqlens=None,
     ``final_state_dtype`` is given. ``out`` may be passed preallocated.
     Returns (out, final_state or None).
     """
+    return _fwd("kda_fwd", q, k, v, g, beta, scale, cu_seqlens, initial_state, final_state, out,
+                final_state_dtype, stream)
+
+
+def kda_fwd_noalloc(q, k, v, g, beta, out, scale: float | None = None, cu_seqlens=None,
+                    initial_state=None, final_state=None, stream=None):
+    """``kda_fwd`` through the allocation-free entry point of include/kda.h.
+
+    The caller provides ``out`` (and ``final_state`` if the final states are
+    wanted): neither this wrapper nor the library allocates. At most
+    ``NOALLOC_MAX_UNITS`` (sequence, head) pairs per call; calls whose work
+    overlaps in time race on the library's fixed scratch. Returns
+    (out, final_state or None).
+    """
+    if out is None:
+        raise ValueError("kda_fwd_noalloc needs a preallocated out tensor")
+    return _fwd("kda_fwd_noalloc", q, k, v, g, beta, scale, cu_seqlens, initial_state, final_state,
+                out, None, stream)
+
+
+def _fwd(entry, q, k, v, g, beta, scale, cu_seqlens, initial_state, final_state, out,
+         final_state_dtype, stream):
     import torch
     _check("q", q, torch.bfloat16, 4)
     _check("k", k, torch.bfloat16, 4)
@@ -139,11 +166,11 @@ def kda_fwd(q, k, v, g, beta, scale: float | None = None, cu_seqlens=None,
         stream = torch.cuda.current_stream(q.device).cuda_stream
     lib = load_library()
     ic, fc = _dtype_code(initial_state), _dtype_code(final_state)
-    st = lib.kda_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(cu_seqlens),
-                     int(N), int(B), int(T), int(H), int(Dk), int(Dv),
-                     _ptr(initial_state), ic if ic >= 0 else 99,
-                     _ptr(final_state), fc if fc >= 0 else 99,
-                     _ptr(out), ctypes.c_void_p(int(stream)))
+    st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                             _ptr(cu_seqlens), int(N), int(B), int(T), int(H), int(Dk), int(Dv),
+                             _ptr(initial_state), ic if ic >= 0 else 99,
+                             _ptr(final_state), fc if fc >= 0 else 99,
+                             _ptr(out), ctypes.c_void_p(int(stream)))
     if st != 0:
         raise KdaError(st, lib.kda_status_string(st).decode())
     return out, final_state

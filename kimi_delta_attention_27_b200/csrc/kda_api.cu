@@ -4,6 +4,8 @@
 #include "../../include/kda.h"
 #include "kda_internal.h"
 
+static_assert(kda::kNoAllocMaxUnits == KDA_NOALLOC_MAX_UNITS, "scratch limit of kda_fwd_noalloc");
+
 namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -20,34 +22,14 @@ bool device_is_sm100(int *err) {
     return major == 10;
 }
 
-}  // namespace
-
-extern "C" {
-
-const char *kda_status_string(kda_status s) {
-    switch (s) {
-        case KDA_OK: return "KDA_OK";
-        case KDA_ERR_NULL_PTR: return "KDA_ERR_NULL_PTR: a required pointer is NULL";
-        case KDA_ERR_BAD_SHAPE: return "KDA_ERR_BAD_SHAPE: head dims must be 128 and sizes non-negative";
-        case KDA_ERR_VARLEN_BATCH: return "KDA_ERR_VARLEN_BATCH: cu_seqlens requires batch == 1";
-        case KDA_ERR_STATE_DTYPE: return "KDA_ERR_STATE_DTYPE: states must be bf16 or fp32 and match";
-        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call failed";
-        case KDA_ERR_UNSUPPORTED_DEVICE: return "KDA_ERR_UNSUPPORTED_DEVICE: needs an sm_100 (B200) device";
-        case KDA_ERR_BAD_ALIGNMENT: return "KDA_ERR_BAD_ALIGNMENT: tensor pointers must be 16-byte aligned";
-        case KDA_ERR_TOO_LARGE: return "KDA_ERR_TOO_LARGE: sizes exceed the library's index range";
-        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a kernel gave up waiting on a barrier and stopped";
-    }
-    return "KDA_ERR_UNKNOWN";
-}
-
-int32_t kda_version(void) { return (1 << 16) | 0; }
-
-kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
-                   const float *beta, float scale, const int32_t *cu_seqlens,
-                   int32_t num_seqs, int32_t batch, int64_t seq_len, int32_t num_heads,
-                   int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
-                   kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype,
-                   void *out, kda_stream_t stream) {
+// Validate the arguments of kda_fwd / kda_fwd_noalloc and fill the kernel parameters.
+// Returns KDA_OK with p->num_seqs == 0 when there is nothing to do.
+kda_status prepare(const void *q, const void *k, const void *v, const float *g, const float *beta, float scale,
+                   const int32_t *cu_seqlens, int32_t num_seqs, int32_t batch, int64_t seq_len,
+                   int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
+                   kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype, void *out,
+                   bool noalloc, kda::FwdParams *p, int64_t *rows_out) {
+    p->num_seqs = 0;
     if (head_dim_k != kda::kHeadDim || head_dim_v != kda::kHeadDim) return KDA_ERR_BAD_SHAPE;
     if (batch < 0 || seq_len < 0 || num_heads < 1 || num_seqs < 0) return KDA_ERR_BAD_SHAPE;
     if (cu_seqlens && batch != 1) return KDA_ERR_VARLEN_BATCH;
@@ -67,28 +49,84 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
     // token offsets are formed as (row * H + h) * 128 in 64-bit; keep the product well inside
     if (rows > (int64_t(1) << 40) / (int64_t(num_heads) * kda::kHeadDim)) return KDA_ERR_TOO_LARGE;
     if (n_seqs * num_heads > (int64_t(1) << 29)) return KDA_ERR_TOO_LARGE;
+    if (noalloc && n_seqs * num_heads > kda::kNoAllocMaxUnits) return KDA_ERR_NOALLOC_LIMIT;
     if (n_seqs == 0) return KDA_OK;
 
     int qerr = 0;
     if (!device_is_sm100(&qerr)) return qerr ? KDA_ERR_CUDA : KDA_ERR_UNSUPPORTED_DEVICE;
 
+    p->q = static_cast<const uint16_t *>(q);
+    p->k = static_cast<const uint16_t *>(k);
+    p->v = static_cast<const uint16_t *>(v);
+    p->g = g;
+    p->beta = beta;
+    p->scale = scale;
+    p->cu_seqlens = cu_seqlens;
+    p->seq_len = seq_len;
+    p->num_seqs = static_cast<int32_t>(n_seqs);
+    p->num_heads = num_heads;
+    p->h0 = initial_state;
+    p->h0_fp32 = initial_dtype == KDA_DTYPE_FP32;
+    p->hT = final_state;
+    p->hT_fp32 = final_dtype == KDA_DTYPE_FP32;
+    p->out = static_cast<uint16_t *>(out);
+    *rows_out = rows;
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_NULL_PTR: return "KDA_ERR_NULL_PTR: a required pointer is NULL";
+        case KDA_ERR_BAD_SHAPE: return "KDA_ERR_BAD_SHAPE: head dims must be 128 and sizes non-negative";
+        case KDA_ERR_VARLEN_BATCH: return "KDA_ERR_VARLEN_BATCH: cu_seqlens requires batch == 1";
+        case KDA_ERR_STATE_DTYPE: return "KDA_ERR_STATE_DTYPE: states must be bf16 or fp32 and match";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call failed";
+        case KDA_ERR_UNSUPPORTED_DEVICE: return "KDA_ERR_UNSUPPORTED_DEVICE: needs an sm_100 (B200) device";
+        case KDA_ERR_BAD_ALIGNMENT: return "KDA_ERR_BAD_ALIGNMENT: tensor pointers must be 16-byte aligned";
+        case KDA_ERR_TOO_LARGE: return "KDA_ERR_TOO_LARGE: sizes exceed the library's index range";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a kernel gave up waiting on a barrier and stopped";
+        case KDA_ERR_NOALLOC_LIMIT:
+            return "KDA_ERR_NOALLOC_LIMIT: kda_fwd_noalloc takes at most 32 (sequence, head) pairs per call";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+int32_t kda_version(void) { return (1 << 16) | 1; }
+
+kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, float scale, const int32_t *cu_seqlens,
+                   int32_t num_seqs, int32_t batch, int64_t seq_len, int32_t num_heads,
+                   int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
+                   kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype,
+                   void *out, kda_stream_t stream) {
     kda::FwdParams p;
-    p.q = static_cast<const uint16_t *>(q);
-    p.k = static_cast<const uint16_t *>(k);
-    p.v = static_cast<const uint16_t *>(v);
-    p.g = g;
-    p.beta = beta;
-    p.scale = scale;
-    p.cu_seqlens = cu_seqlens;
-    p.seq_len = seq_len;
-    p.num_seqs = static_cast<int32_t>(n_seqs);
-    p.num_heads = num_heads;
-    p.h0 = initial_state;
-    p.h0_fp32 = initial_dtype == KDA_DTYPE_FP32;
-    p.hT = final_state;
-    p.hT_fp32 = final_dtype == KDA_DTYPE_FP32;
-    p.out = static_cast<uint16_t *>(out);
+    int64_t rows = 0;
+    const kda_status st = prepare(q, k, v, g, beta, scale, cu_seqlens, num_seqs, batch, seq_len, num_heads,
+                                  head_dim_k, head_dim_v, initial_state, initial_dtype, final_state,
+                                  final_dtype, out, false, &p, &rows);
+    if (st != KDA_OK || p.num_seqs == 0) return st;
     const cudaError_t err = kda::launch_fwd_tc(p, rows, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_fwd_noalloc(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, float scale, const int32_t *cu_seqlens,
+                           int32_t num_seqs, int32_t batch, int64_t seq_len, int32_t num_heads,
+                           int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
+                           kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype,
+                           void *out, kda_stream_t stream) {
+    kda::FwdParams p;
+    int64_t rows = 0;
+    const kda_status st = prepare(q, k, v, g, beta, scale, cu_seqlens, num_seqs, batch, seq_len, num_heads,
+                                  head_dim_k, head_dim_v, initial_state, initial_dtype, final_state,
+                                  final_dtype, out, true, &p, &rows);
+    if (st != KDA_OK || p.num_seqs == 0) return st;
+    const cudaError_t err = kda::launch_fwd_tc_noalloc(p, rows, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -240,6 +240,13 @@ __device__ __forceinline__ uint32_t smid() {
     return r;
 }
 
+// kRingPerCluster == false: `rings` holds kMaxRings rings and a cluster uses the one of
+// its chain CTA's SM (a chain CTA fills an SM's shared memory, so no two resident
+// clusters, of this launch or of any other, share a ring).
+// kRingPerCluster == true: `rings` holds one ring per cluster of this launch and
+// cluster c uses ring c (the allocation-free entry point, whose fixed scratch bounds
+// the cluster count).
+template <bool kRingPerCluster>
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_fwd_tc_kernel(const FwdParams p, const __grid_constant__ TmaMaps maps, unsigned char *rings) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -308,10 +315,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     cluster_wait();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(miscg + M_TMEM);
-    // this cluster's ring: indexed by the chain CTA's SM (unique among resident clusters)
-    const uint32_t ring_id = is_chain ? *reinterpret_cast<volatile uint32_t *>(miscg + M_SMID)
-                                      : ld_shared_cluster_u32(mapa(sbase + CH_MISC + M_SMID, 0));
-    if (!is_chain && ring_id >= static_cast<uint32_t>(kMaxRings) && tid == 0) *abort_flag = 1;
+    uint32_t ring_id;
+    if constexpr (kRingPerCluster) {
+        ring_id = blockIdx.x / NS;
+    } else {
+        // this cluster's ring: indexed by the chain CTA's SM (unique among resident clusters)
+        ring_id = is_chain ? *reinterpret_cast<volatile uint32_t *>(miscg + M_SMID)
+                           : ld_shared_cluster_u32(mapa(sbase + CH_MISC + M_SMID, 0));
+        if (!is_chain && ring_id >= static_cast<uint32_t>(kMaxRings) && tid == 0) *abort_flag = 1;
+    }
     unsigned char *ring = rings + static_cast<uint64_t>(ring_id < kMaxRings ? ring_id : 0) * RING_BYTES;
 
     if (is_chain) {
@@ -1083,18 +1095,34 @@ unsigned char *ring_pool(int dev) {
     return g_pool[dev];
 }
 
-}  // namespace
+// Scratch of the allocation-free entry point: one operand-set ring per cluster for at
+// most kNoAllocMaxUnits clusters (15.4 MiB). It is part of the module image, so it
+// exists as soon as the module is loaded and nothing is allocated when it is used.
+// Nothing in it has to start at zero: a prep CTA writes every ring slot before it
+// signals the chain CTA to read it.
+static __device__ __align__(256) unsigned char g_noalloc_rings[kNoAllocMaxUnits * tc::RING_BYTES];
 
-cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream) {
-    const int64_t units = static_cast<int64_t>(p.num_seqs) * p.num_heads;
-    if (units == 0) return cudaSuccess;
-    const int64_t grid = units * tc::NS;
-    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess) return err;
-    unsigned char *rings = ring_pool(dev);
-    if (!rings) return cudaErrorMemoryAllocation;
+std::mutex g_noalloc_mu;
+unsigned char *g_noalloc_addr[64] = {};
+
+// Device address of g_noalloc_rings on `dev` (the current device), looked up once.
+cudaError_t noalloc_scratch(int dev, unsigned char **out) {
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *ptr = nullptr;
+        const cudaError_t err = cudaGetSymbolAddress(&ptr, g_noalloc_rings);
+        if (err != cudaSuccess) return err;
+        g_noalloc_addr[dev] = static_cast<unsigned char *>(ptr);
+    }
+    *out = g_noalloc_addr[dev];
+    return cudaSuccess;
+}
+
+// Encode the tensor maps and launch one 4-CTA cluster per (sequence, head).
+template <bool kRingPerCluster>
+cudaError_t launch_clusters(const FwdParams &p, int64_t rows, int64_t grid, unsigned char *rings,
+                            cudaStream_t stream) {
     tc::TmaMaps maps;
     memset(&maps, 0, sizeof(maps));
     if (rows > 0) {
@@ -1111,8 +1139,9 @@ cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream)
                       CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
-    err = cudaFuncSetAttribute(tc::kda_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(tc::SMEM_BYTES));
+    cudaError_t err = cudaFuncSetAttribute(tc::kda_fwd_tc_kernel<kRingPerCluster>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(tc::SMEM_BYTES));
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
@@ -1126,9 +1155,37 @@ cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, tc::kda_fwd_tc_kernel, p, maps, rings);
+    err = cudaLaunchKernelEx(&cfg, tc::kda_fwd_tc_kernel<kRingPerCluster>, p, maps, rings);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream) {
+    const int64_t units = static_cast<int64_t>(p.num_seqs) * p.num_heads;
+    if (units == 0) return cudaSuccess;
+    const int64_t grid = units * tc::NS;
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    unsigned char *rings = ring_pool(dev);
+    if (!rings) return cudaErrorMemoryAllocation;
+    return launch_clusters<false>(p, rows, grid, rings, stream);
+}
+
+cudaError_t launch_fwd_tc_noalloc(const FwdParams &p, int64_t rows, cudaStream_t stream) {
+    const int64_t units = static_cast<int64_t>(p.num_seqs) * p.num_heads;
+    if (units == 0) return cudaSuccess;
+    if (units > kNoAllocMaxUnits) return cudaErrorInvalidValue;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    unsigned char *rings = nullptr;
+    err = noalloc_scratch(dev, &rings);
+    if (err != cudaSuccess) return err;
+    return launch_clusters<true>(p, rows, units * tc::NS, rings, stream);
 }
 
 #ifdef KDA_TRACE

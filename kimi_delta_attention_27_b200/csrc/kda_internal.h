@@ -32,6 +32,12 @@ cudaError_t launch_fwd_simt(const FwdParams &p, cudaStream_t stream);
 // number of token rows of the packed [rows, H, 128] tensors.
 cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream);
 
+// Allocation-free variant of launch_fwd_tc: the operand-set rings live in a fixed
+// module-scope array, one per cluster, so at most kNoAllocMaxUnits (sequence, head)
+// pairs are accepted per call (cudaErrorInvalidValue beyond that).
+constexpr int kNoAllocMaxUnits = 32;
+cudaError_t launch_fwd_tc_noalloc(const FwdParams &p, int64_t rows, cudaStream_t stream);
+
 // Device-side error word of the tensor-core kernel (bit 0: a bounded wait gave up).
 cudaError_t read_and_clear_device_error(unsigned int *value);
 
