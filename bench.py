@@ -63,13 +63,16 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+# the sources the timed kernel is compiled from
+KERNEL_SOURCES = ("kda_fwd_tc.cu", "kda_internal.h", "sm100_ptx.cuh")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kimi_delta_attention_27_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode()); h.update(f.read())
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode()); h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -154,13 +157,26 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of every rank's ``x`` (the slowest rank's time)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_value(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Tokens/s of the whole job: every rank's tokens over the slowest rank's step time."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Seed of rank ``rank``'s workload: each rank processes its own independent
+    batch (weak scaling), never a copy of another rank's."""
+    return base_seed + 1000 * rank
 
 
 def cpu_baseline_run(inp, tokens_per_step, steps=1, warmup=0):
@@ -269,7 +285,7 @@ def main():
 
     name = args.workload
     cfg = dict(CONFIGS[name])
-    inp = make_inputs(name, device="cuda", seed=cfg["seed"] + 1000 * rank)
+    inp = make_inputs(name, device="cuda", seed=rank_seed(cfg["seed"], rank))
     H, N, tokens = inp["H"], inp["N"], inp["B"] * inp["T"]
     final_dt = inp["final_dtype"]
     out = torch.empty_like(inp["v"])
@@ -313,7 +329,7 @@ def main():
     total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
     ms_per_step = total_ms / args.steps
-    value = world * tokens / (ms_per_step / 1e3)
+    value = whole_job_value(world, tokens, ms_per_step)
     flops = pages_flops(tokens, H)
     peaks = load_peaks()
     alg_bytes = tokens * H * BYTES_PER_TOKEN_HEAD + state_bytes(

@@ -25,9 +25,6 @@ struct FwdParams {
     uint16_t *out;              // bf16 [rows, H, 128]
 };
 
-// First, straightforward CUDA-core path (fp32 arithmetic throughout).
-cudaError_t launch_fwd_simt(const FwdParams &p, cudaStream_t stream);
-
 // Tensor-core path: one 4-CTA cluster per (sequence, head); `rows` is the
 // number of token rows of the packed [rows, H, 128] tensors.
 cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream);
