@@ -53,14 +53,24 @@ __device__ unsigned int g_kda_device_error = 0;
 #ifdef KDA_TRACE
 // Development-only timeline: when built with -DKDA_TRACE, the first cluster
 // records %globaltimer at fixed points per chunk into g_kda_trace
-// [rank][chunk < 64][point < 16]. The product build compiles none of this.
-__device__ unsigned long long g_kda_trace[4 * 64 * 16];
+// [rank][chunk < 64][point < 32]. The product build compiles none of this.
+__device__ unsigned long long g_kda_trace[4 * 64 * 32];
+// per cluster: chain CTA start, end, SM id, then the SM ids of ranks 1-3 and the ring address
+__device__ unsigned long long g_kda_cluster_trace[1024 * 8];
+#define KDA_TRACE_CLUSTER(slot, value)                                                              \
+    do {                                                                                            \
+        if (blockIdx.x / 4 < 1024) g_kda_cluster_trace[(blockIdx.x / 4) * 8 + (slot)] = (value);    \
+    } while (0)
+__device__ int g_kda_trace_cluster = 0;   // the cluster whose chunks are timed
 #define KDA_TRACE_POINT(chunk, point)                                                               \
     do {                                                                                            \
-        if (blockIdx.x < 4 && (chunk) < 64)                                                         \
-            g_kda_trace[(rank * 64 + (chunk)) * 16 + (point)] = ptx::globaltimer();                 \
+        if (static_cast<int>(blockIdx.x / 4) == g_kda_trace_cluster && (chunk) < 64)                \
+            g_kda_trace[(rank * 64 + (chunk)) * 32 + (point)] = ptx::globaltimer();                 \
     } while (0)
 #else
+#define KDA_TRACE_CLUSTER(slot, value) \
+    do {                               \
+    } while (0)
 #define KDA_TRACE_POINT(chunk, point) \
     do {                              \
     } while (0)
@@ -109,7 +119,7 @@ static_assert(PR_AVT % 1024 == 0 && PR_WP % 1024 == 0 && CH_SP % 1024 == 0 && PR
 
 // misc area (offsets from the misc base of either role)
 constexpr uint32_t M_BAR = 0;                      // up to 32 barriers
-constexpr uint32_t M_BETA = 256, M_EGA = 512, M_GSUM = 1024;   // 64, 128, 2 x 128 floats
+constexpr uint32_t M_BETA = 256, M_EGA = 512;                  // 64, 128 floats
 constexpr uint32_t M_DEC = 2048;                               // 2 x 128 floats (e^Gl, part of the set)
 constexpr uint32_t M_TMEM = 3072, M_ABORT = 3088, M_SMID = 3104;
 constexpr uint32_t MISC_BYTES = 3584;
@@ -119,8 +129,8 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 // chain barriers
 enum {
     CB_FULL = 0,     // 2: operand set landed in smem slot (1 arrival + tx)
-    CB_SFREE = 2,    // 2: smem slot consumed (8 epilogue warps + the output store warp)
-    CB_C1_FULL = 4, CB_C1_FREE, CB_S_READY, CB_D_READY, CB_C3_FULL,
+    CB_SFREE = 2,    // 2: smem slot consumed (8 epilogue warps, the output store warp, the release warp)
+    CB_C1_FULL = 4, CB_C3_FULL = 8,
     CB_O_READY = 9,  // output tile staged in the slot (4 warps)
     CB_READY = 10,   // 6: ring slot written by a prep CTA (remote arrival)
     CB_COUNT = 16
@@ -184,6 +194,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
     __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&h);
+}
+
+constexpr float kLog2e = 1.4426950408889634f;   // log2(e)
+
+// 2^y by the hardware approximation (relative error about 2^-22; subnormal results flush to 0)
+__device__ __forceinline__ float ex2_approx(float y) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y));
+    return r;
 }
 
 // byte offset of 16-byte chunk j of row r in a tile of 128-byte rows, 128B swizzle
@@ -285,12 +304,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (is_chain) {
             for (int i = 0; i < 2; ++i) {
                 mbar_init(BAR(CB_FULL + i), 1);
-                mbar_init(BAR(CB_SFREE + i), 9);
+                mbar_init(BAR(CB_SFREE + i), 10);
             }
             mbar_init(BAR(CB_C1_FULL), 1);
-            mbar_init(BAR(CB_C1_FREE), 8);
-            mbar_init(BAR(CB_S_READY), 8);
-            mbar_init(BAR(CB_D_READY), 4);
             mbar_init(BAR(CB_C3_FULL), 1);
             mbar_init(BAR(CB_O_READY), 4);
             for (int i = 0; i < NRING; ++i) mbar_init(BAR(CB_READY + i), 1);
@@ -326,6 +342,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     unsigned char *ring = rings + static_cast<uint64_t>(ring_id < kMaxRings ? ring_id : 0) * RING_BYTES;
 
+    if (tid == 0) {
+        if (is_chain) {
+            KDA_TRACE_CLUSTER(0, globaltimer());
+            KDA_TRACE_CLUSTER(7, static_cast<unsigned long long>(clock64()));
+        }
+        KDA_TRACE_CLUSTER(2 + rank, smid());
+    }
     if (is_chain) {
         // ======================================================================= chain CTA
         if (warp == 0) {
@@ -373,41 +396,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 __syncwarp();
             }
-        } else if (warp == 1) {
-            // ---- chain MMA issuer
+        } else if (warp == 3) {
+            // ---- ring slot release: once chunk n's set has landed in shared memory, its ring
+            // slot goes back to the producer of chunk n + NRING. A cluster-scope remote arrival
+            // can hold the issuing thread for a while, so it is kept off the MMA warp.
             for (int n = 0; n < nch; ++n) {
                 const int sl = n & 1;
-                const uint32_t slot = sbase + CH_SLOT + sl * SET_STRIDE;
                 if (!wait_bar(BAR(CB_FULL + sl), (n >> 1) & 1, abort_flag)) break;
-                if (lane == 0) KDA_TRACE_POINT(n, 12);
-                // the ring slot has been copied out: hand it back to the producer of chunk n + NRING
-                if (lane == 0 && n + NRING < nch) {
-                    const uint32_t prod = 1u + static_cast<uint32_t>(n % NPREP);
-                    mbar_arrive_remote(mapa(sbase + PR_MISC + M_BAR + 8u * (PB_RING_FREE + n % NRING), prod));
-                }
-                if (n >= 1 && !wait_bar(BAR(CB_C1_FREE), (n - 1) & 1, abort_flag)) break;
-                if (!wait_bar(BAR(CB_S_READY), n & 1, abort_flag)) break;
-                tc_fence_after();
                 if (lane == 0) {
-                    KDA_TRACE_POINT(n, 13);
-                    // state part: [-W; Qt] * S'   (bf16)
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_f16(tmem + COL_C1, smem_desc(slot + SET_W + ks * 2048, 16384, 1024, kSwizzle128),
-                                smem_desc(sbase + CH_SP + ks * 2048, 16384, 1024, kSwizzle128), ID_STATE, ks > 0);
-                    mma_commit(BAR(CB_C1_FULL));
-                    KDA_TRACE_POINT(n, 3);
-                }
-                __syncwarp();
-                if (!wait_bar(BAR(CB_D_READY), n & 1, abort_flag)) break;
-                tc_fence_after();
-                if (lane == 0) KDA_TRACE_POINT(n, 4);
-                if (lane == 0) {
-                    // state increment: Kt^T * D   (fp16)
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tmem + COL_C3, smem_desc(slot + SET_KT + ks * 32, 16, 1024, kSwizzle128),
-                                smem_desc(sbase + CH_DL + ks * 2048, 8192, 1024, kSwizzle128), ID_C3, ks > 0);
-                    mma_commit(BAR(CB_C3_FULL));
-                    KDA_TRACE_POINT(n, 5);
+                    if (n + NRING < nch) {
+                        const uint32_t prod = 1u + static_cast<uint32_t>(n % NPREP);
+                        mbar_arrive_remote(mapa(sbase + PR_MISC + M_BAR + 8u * (PB_RING_FREE + n % NRING), prod));
+                    }
+                    mbar_arrive(BAR(CB_SFREE + sl));
                 }
                 __syncwarp();
             }
@@ -453,10 +454,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                  pack_bf16(S[8 * j + 2], S[8 * j + 3]), pack_bf16(S[8 * j + 4], S[8 * j + 5]),
                                  pack_bf16(S[8 * j + 6], S[8 * j + 7]));
             };
+            // The MMAs are issued by one thread of the epilogue warps as soon as their operands
+            // are in place (a named barrier among the writers), with no hop through another warp:
+            //   C1 = [-W; Qt] S'   (bf16; S' written by all 8 warps)
+            //   C3 = Kt^T D        (fp16; D written by the 4 warps of rows 0..63)
+            auto issue_c1 = [&](int n) -> bool {
+                const int s1 = n & 1;
+                const uint32_t slot = sbase + CH_SLOT + s1 * SET_STRIDE;
+                if (!wait_bar(BAR(CB_FULL + s1), (n >> 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                KDA_TRACE_POINT(n, 13);
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_f16(tmem + COL_C1, smem_desc(slot + SET_W + ks * 2048, 16384, 1024, kSwizzle128),
+                            smem_desc(sbase + CH_SP + ks * 2048, 16384, 1024, kSwizzle128), ID_STATE, ks > 0);
+                mma_commit(BAR(CB_C1_FULL));
+                KDA_TRACE_POINT(n, 3);
+                return true;
+            };
+            auto issue_c3 = [&](int n) {
+                const uint32_t slot = sbase + CH_SLOT + (n & 1) * SET_STRIDE;
+                tc_fence_after();
+                KDA_TRACE_POINT(n, 4);
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tmem + COL_C3, smem_desc(slot + SET_KT + ks * 32, 16, 1024, kSwizzle128),
+                            smem_desc(sbase + CH_DL + ks * 2048, 8192, 1024, kSwizzle128), ID_C3, ks > 0);
+                mma_commit(BAR(CB_C3_FULL));
+                KDA_TRACE_POINT(n, 5);
+            };
             write_sprime();
             fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(4, 256);
+            if (tid == 128 && nch > 0) issue_c1(0);
             __syncwarp();
-            if (lane == 0) mbar_arrive(BAR(CB_S_READY));
             for (int n = 0; n < nch; ++n) {
                 const int sl = n & 1;
                 const int64_t t0 = bos + static_cast<int64_t>(n) * C;
@@ -465,50 +495,63 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_fence_after();
                 if (tid == 128) KDA_TRACE_POINT(n, 9);
                 {
-                    uint32_t r0[32], r1[32];
-                    tmem_ld32(tmem + lane_base + COL_C1 + c0, r0);
-                    tmem_ld32(tmem + lane_base + COL_C1 + c0 + 32, r1);
-                    // value side of this row (U for rows < 64, Aqk U below), fp16
+                    // value side of this row (U for rows < 64, Aqk U below), fp16; the row's 64
+                    // columns are done as two halves so that the TMEM and shared-memory loads of a
+                    // half are in flight together
                     const uint32_t uvb = sbase + CH_SLOT + sl * SET_STRIDE + SET_UV + half * 16384;
-                    tmem_wait_ld();
-                    // x = accumulator + value side, computed 8 columns at a time and stored at once
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint4 u = ld_shared_v4(uvb + sw128(row, j));
-                        const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
-                        uint32_t *rr = j < 4 ? r0 + 8 * j : r1 + 8 * (j - 4);
-                        float x[8];
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t r[32];
+                        tmem_ld32(tmem + lane_base + COL_C1 + c0 + 32 * hh, r);
+                        uint4 u4[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 uf = __half22float2(*reinterpret_cast<const __half2 *>(&uw[e]));
-                            x[2 * e] = __uint_as_float(rr[2 * e]) + uf.x;
-                            x[2 * e + 1] = __uint_as_float(rr[2 * e + 1]) + uf.y;
-                        }
-                        if (row < 64) {
-                            // pseudo-values D -> fp16 B operand of the state increment
-                            st_shared_v4(sbase + CH_DL + half * 8192 + sw128(row, j), pack_f16(x[0], x[1]),
-                                         pack_f16(x[2], x[3]), pack_f16(x[4], x[5]), pack_f16(x[6], x[7]));
-                        } else {
-                            // output row -> staging tile over the value-side rows just consumed
-                            // (same bytes this thread read above); the store warp writes it out
-                            const float sc = p.scale;
-                            st_shared_v4(uvb + sw128(row, j), pack_bf16(sc * x[0], sc * x[1]),
-                                         pack_bf16(sc * x[2], sc * x[3]), pack_bf16(sc * x[4], sc * x[5]),
-                                         pack_bf16(sc * x[6], sc * x[7]));
+                        for (int j = 0; j < 4; ++j) u4[j] = ld_shared_v4(uvb + sw128(row, 4 * hh + j));
+                        tmem_wait_ld();
+                        if (tid == 128 && hh == 0) KDA_TRACE_POINT(n, 0);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t uw[4] = {u4[j].x, u4[j].y, u4[j].z, u4[j].w};
+                            const uint32_t *rr = r + 8 * j;
+                            float x[8];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 uf = __half22float2(*reinterpret_cast<const __half2 *>(&uw[e]));
+                                x[2 * e] = __uint_as_float(rr[2 * e]) + uf.x;
+                                x[2 * e + 1] = __uint_as_float(rr[2 * e + 1]) + uf.y;
+                            }
+                            const int jj = 4 * hh + j;
+                            if (row < 64) {
+                                // pseudo-values D -> fp16 B operand of the state increment
+                                st_shared_v4(sbase + CH_DL + half * 8192 + sw128(row, jj), pack_f16(x[0], x[1]),
+                                             pack_f16(x[2], x[3]), pack_f16(x[4], x[5]), pack_f16(x[6], x[7]));
+                            } else {
+                                // output row -> staging tile over the value-side rows just consumed
+                                // (same bytes this thread read above); the store warp writes it out
+                                const float sc = p.scale;
+                                st_shared_v4(uvb + sw128(row, jj), pack_bf16(sc * x[0], sc * x[1]),
+                                             pack_bf16(sc * x[2], sc * x[3]), pack_bf16(sc * x[4], sc * x[5]),
+                                             pack_bf16(sc * x[6], sc * x[7]));
+                            }
                         }
                     }
+                    if (tid == 128) KDA_TRACE_POINT(n, 1);
                     fence_proxy_async_smem();
+                    if (tid == 128) KDA_TRACE_POINT(n, 2);
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (tid == 128) KDA_TRACE_POINT(n, 6);
-                if (lane == 0) {
-                    mbar_arrive(BAR(CB_C1_FREE));
-                    mbar_arrive(BAR(row < 64 ? CB_D_READY : CB_O_READY));
+                if (row < 64) {
+                    named_bar_sync(3, 128);
+                    if (tid == 128) issue_c3(n);
+                    __syncwarp();
+                } else if (lane == 0) {
+                    mbar_arrive(BAR(CB_O_READY));
                 }
                 if (!wait_bar(BAR(CB_C3_FULL), n & 1, abort_flag)) break;
                 tc_fence_after();
                 if (tid == 128) KDA_TRACE_POINT(n, 10);
+                if (lane == 0) KDA_TRACE_POINT(n, 24 + warp - 4);
                 {
                     uint32_t r0[32], r1[32];
                     tmem_ld32(tmem + lane_base + COL_C3 + c0, r0);
@@ -524,15 +567,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (tid == 128) KDA_TRACE_POINT(n, 8);
                 if (n + 1 < nch) {
                     write_sprime();
+                    if (tid == 128) KDA_TRACE_POINT(n, 7);
                     fence_proxy_async_smem();
+                    if (tid == 128) KDA_TRACE_POINT(n, 14);
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    if (n + 1 < nch) mbar_arrive(BAR(CB_S_READY));
-                    mbar_arrive(BAR(CB_SFREE + sl));
+                if (lane == 0) mbar_arrive(BAR(CB_SFREE + sl));
+                if (n + 1 < nch) {
+                    named_bar_sync(4, 256);
+                    bool ok = true;
+                    if (tid == 128) ok = issue_c1(n + 1);
+                    __syncwarp();
+                    if (!ok) break;
                 }
                 if (tid == 128) KDA_TRACE_POINT(n, 11);
+                if (lane == 0) KDA_TRACE_POINT(n, 16 + warp - 4);
             }
             // final state
             if (p.hT && !*abort_flag) {
@@ -629,29 +679,36 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 unsigned char *set = ring + static_cast<uint64_t>(r) * SET_STRIDE;
                 // the ring slot must have been pulled by the chain CTA (chunk m - NRING)
                 if (m >= NRING && !wait_bar(BAR(PB_RING_FREE + r), ((m / NRING) - 1) & 1, abort_flag)) break;
+                if (lane == 0) KDA_TRACE_POINT(m, 18);
                 if (!wait_bar(BAR(PB_OUTA_READY), kk & 1, abort_flag)) break;
                 if (lane == 0) {
+                    KDA_TRACE_POINT(m, 19);
                     bulk_s2g(set + SET_KT, sbase + PR_KC, 16384);
                     bulk_commit();
                 }
                 __syncwarp();
                 if (!wait_bar(BAR(PB_OUTB_READY), kk & 1, abort_flag)) break;
                 if (lane == 0) {
+                    KDA_TRACE_POINT(m, 20);
                     bulk_s2g(set + SET_W, sbase + PR_KH, 16384);
                     bulk_commit();
                     bulk_wait_read0();
+                    KDA_TRACE_POINT(m, 21);
                     mbar_arrive(BAR(PB_OUTAB_FREE));
                 }
                 __syncwarp();
                 if (!wait_bar(BAR(PB_OUTC_READY), kk & 1, abort_flag)) break;
                 if (lane == 0) {
+                    KDA_TRACE_POINT(m, 22);
                     bulk_s2g(set + SET_Q, sbase + PR_AVT, 16384);
                     bulk_s2g(set + SET_UV, sbase + PR_AKK, 32768);
                     bulk_s2g(set + SET_DEC, misc + M_DEC + (kk & 1) * 512, 512);
                     bulk_commit();
                     bulk_wait_read0();
+                    KDA_TRACE_POINT(m, 23);
                     mbar_arrive(BAR(PB_OUTC_FREE));
                     bulk_wait0();
+                    KDA_TRACE_POINT(m, 24);
                     fence_proxy_async_global();
                     mbar_arrive_remote(mapa(sbase + CH_MISC + M_BAR + 8u * (CB_READY + r), 0));
                     KDA_TRACE_POINT(m, 8);
@@ -668,74 +725,120 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             float *wsf = reinterpret_cast<float *>(sgen);
             float *beta_s = reinterpret_cast<float *>(miscg + M_BETA);
             float *ega_s = reinterpret_cast<float *>(miscg + M_EGA);
-            float *gsum = reinterpret_cast<float *>(miscg + M_GSUM);
             float *dec_all = reinterpret_cast<float *>(miscg + M_DEC);
+            // beta of chunk m (0 past the sequence end), loaded one chunk of this CTA ahead so
+            // that its global-memory latency is hidden behind the previous chunk's work
+            auto load_beta = [&](int m) -> float {
+                const int64_t tok = bos + static_cast<int64_t>(m) * C + t;
+                return (t < C && m < nch && tok < eos) ? p.beta[tok * H + h] : 0.f;
+            };
+            float beta_next = load_beta(first);
             int kk = 0;
             for (int m = first; m < nch; m += NPREP, ++kk) {
                 const int64_t t0 = bos + static_cast<int64_t>(m) * C;
                 const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
                 if (*abort_flag) break;
                 if (t == 0) KDA_TRACE_POINT(m, 0);
-                if (t < C) beta_s[t] = t < L ? p.beta[(t0 + t) * H + h] : 0.f;
+                if (t < C) beta_s[t] = beta_next;
+                beta_next = load_beta(m + NPREP);
                 // parts A and B of the previous set must have been read out by the publisher
                 if (kk >= 1 && !wait_bar(BAR(PB_OUTAB_FREE), (kk - 1) & 1, abort_flag)) break;
                 if (!wait_bar(BAR(PB_STAGE_FULL), kk & 1, abort_flag)) break;
                 if (t == 0) KDA_TRACE_POINT(m, 1);
 
-                // -------- S1: running log-decay, two threads per channel (rows 0-31 / 32-63)
-                uint32_t ktr[16];   // Kt^T row of this thread (fp16 pairs), stored after the S2 MMA
+                // -------- S1: running log-decay and the anchored factors. A thread owns a pair of
+                // adjacent channels (c0, c0 + 1) over one quarter of the rows (16 tokens), so q and k
+                // are read as bf16 pairs and g as float pairs.
+                uint32_t ktr[16];   // Kt^T of this thread: 4 fp16 pairs x 2 chunks x 2 channels
                 {
-                    const int c = t & 127, hr = t >> 7;
-                    const float *gcol = reinterpret_cast<const float *>(sgen + PR_STG + STG_G) + c;
-                    const uint16_t *qcol = reinterpret_cast<const uint16_t *>(sgen + PR_STG + STG_Q) + c;
-                    const uint16_t *kcol = reinterpret_cast<const uint16_t *>(sgen + PR_STG + STG_K) + c;
-                    float gv[32];
-                    float part = 0.f;
+                    const int grp = (warp - 4) & 3;
+                    const int cp = grp * 16 + (lane & 15);
+                    const int tq = 2 * ((warp - 4) >> 2) + (lane >> 4);
+                    const int c0 = 2 * cp, r0 = 16 * tq;
+                    const float *gst = reinterpret_cast<const float *>(sgen + PR_STG + STG_G);
+                    const uint32_t *qst = reinterpret_cast<const uint32_t *>(sgen + PR_STG + STG_Q);
+                    const uint32_t *kst = reinterpret_cast<const uint32_t *>(sgen + PR_STG + STG_K);
+                    float2 gv[16];
+                    float px = 0.f, py = 0.f;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int rr = hr * 32 + i;
-                        gv[i] = rr < L ? gcol[rr * D] : 0.f;
-                        part += gv[i];
+                    for (int i = 0; i < 16; ++i) {
+                        const int rr = r0 + i;
+                        gv[i] = rr < L ? *reinterpret_cast<const float2 *>(gst + rr * D + c0) : make_float2(0.f, 0.f);
+                        px += gv[i].x;
+                        py += gv[i].y;
                     }
-                    gsum[hr * 128 + c] = part;
+                    // row-quarter sums of g per channel, [4][128] floats in the solve's scratch
+                    float *gq = reinterpret_cast<float *>(sgen + PR_P);
+                    *reinterpret_cast<float2 *>(gq + tq * 128 + c0) = make_float2(px, py);
                     named_bar_sync(2, 256);
-                    const float ga = gsum[c];                   // G at the anchor row 31
-                    const float gl = ga + gsum[128 + c];        // G at the last row
-                    const float eca = __expf(gl - ga);
-                    float G = hr ? ga : 0.f;
+                    float2 qs[4];
 #pragma unroll
-                    for (int rb = 0; rb < 4; ++rb) {
-                        uint32_t ph[4], pq[4], pc[4];
+                    for (int q = 0; q < 4; ++q) qs[q] = *reinterpret_cast<const float2 *>(gq + q * 128 + c0);
+                    const float gax = qs[0].x + qs[1].x, gay = qs[0].y + qs[1].y;   // G at the anchor row 31
+                    const float glx = gax + qs[2].x + qs[3].x, gly = gay + qs[2].y + qs[3].y;   // G at row 63
+                    float Gx = 0.f, Gy = 0.f;                                        // G before row r0
+#pragma unroll
+                    for (int q = 0; q < 3; ++q)
+                        if (q < tq) {
+                            Gx += qs[q].x;
+                            Gy += qs[q].y;
+                        }
+                    const float ecx = ex2_approx(kLog2e * (glx - gax)), ecy = ex2_approx(kLog2e * (gly - gay));
+                    // the channel pair is written as two rows; lanes 4-7 of every 8 write the odd
+                    // channel first, so that one store instruction covers all eight swizzle phases
+                    const bool odd_first = (lane >> 2) & 1;
+#pragma unroll
+                    for (int h8 = 0; h8 < 2; ++h8) {
+                        uint32_t hx[4], hy[4], qx4[4], qy4[4], cx[4], cy[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            float kh[2], qh[2], kc[2], kt[2];
+                            float khx[2], khy[2], qhx[2], qhy[2], kcx[2], kcy[2], ktx[2], kty[2];
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
-                                const int i = rb * 8 + 2 * e + u, rr = hr * 32 + i;
-                                const bool valid = rr < L;
-                                G += gv[i];
-                                const float x = G - ga;
-                                const float ep = __expf(x), em = __expf(-x);
-                                const float kv = valid ? bf2f(kcol[rr * D]) : 0.f;
-                                const float qv = valid ? bf2f(qcol[rr * D]) : 0.f;
-                                kh[u] = kv * ep;
-                                qh[u] = qv * ep;
-                                kc[u] = kv * em;
-                                kt[u] = kc[u] * eca;
+                                const int i = h8 * 8 + 2 * e + u, rr = r0 + i;
+                                Gx += gv[i].x;
+                                Gy += gv[i].y;
+                                const float yx = kLog2e * (Gx - gax), yy = kLog2e * (Gy - gay);
+                                const float epx = ex2_approx(yx), emx = ex2_approx(-yx);
+                                const float epy = ex2_approx(yy), emy = ex2_approx(-yy);
+                                const uint32_t kw = rr < L ? kst[rr * (D / 2) + cp] : 0u;
+                                const uint32_t qw = rr < L ? qst[rr * (D / 2) + cp] : 0u;
+                                khx[u] = lo_bf(kw) * epx;
+                                khy[u] = hi_bf(kw) * epy;
+                                qhx[u] = lo_bf(qw) * epx;
+                                qhy[u] = hi_bf(qw) * epy;
+                                kcx[u] = lo_bf(kw) * emx;
+                                kcy[u] = hi_bf(kw) * emy;
+                                ktx[u] = kcx[u] * ecx;
+                                kty[u] = kcy[u] * ecy;
                             }
-                            ph[e] = pack_bf16(kh[0], kh[1]);
-                            pq[e] = pack_bf16(qh[0], qh[1]);
-                            pc[e] = pack_bf16(kc[0], kc[1]);
-                            ktr[rb * 4 + e] = pack_f16(kt[0], kt[1]);
+                            hx[e] = pack_bf16(khx[0], khx[1]);
+                            hy[e] = pack_bf16(khy[0], khy[1]);
+                            qx4[e] = pack_bf16(qhx[0], qhx[1]);
+                            qy4[e] = pack_bf16(qhy[0], qhy[1]);
+                            cx[e] = pack_bf16(kcx[0], kcx[1]);
+                            cy[e] = pack_bf16(kcy[0], kcy[1]);
+                            ktr[h8 * 4 + e] = pack_f16(ktx[0], ktx[1]);
+                            ktr[8 + h8 * 4 + e] = pack_f16(kty[0], kty[1]);
                         }
-                        const uint32_t o = sw128(c, hr * 4 + rb);
-                        st_shared_v4(sbase + PR_KH + o, ph[0], ph[1], ph[2], ph[3]);
-                        st_shared_v4(sbase + PR_QH + o, pq[0], pq[1], pq[2], pq[3]);
-                        st_shared_v4(sbase + PR_KC + o, pc[0], pc[1], pc[2], pc[3]);
+                        const int j = 2 * tq + h8;   // 16-byte chunk (8 tokens) of a channel row
+                        const uint32_t ra = c0 + (odd_first ? 1 : 0), rb2 = c0 + (odd_first ? 0 : 1);
+#pragma unroll
+                        for (int tile = 0; tile < 3; ++tile) {
+                            const uint32_t base = sbase + (tile == 0 ? PR_KH : (tile == 1 ? PR_QH : PR_KC));
+                            const uint32_t *X = tile == 0 ? hx : (tile == 1 ? qx4 : cx);
+                            const uint32_t *Y = tile == 0 ? hy : (tile == 1 ? qy4 : cy);
+                            st_shared_v4(base + sw128(ra, j), odd_first ? Y[0] : X[0], odd_first ? Y[1] : X[1],
+                                         odd_first ? Y[2] : X[2], odd_first ? Y[3] : X[3]);
+                            st_shared_v4(base + sw128(rb2, j), odd_first ? X[0] : Y[0], odd_first ? X[1] : Y[1],
+                                         odd_first ? X[2] : Y[2], odd_first ? X[3] : Y[3]);
+                        }
                     }
-                    if (hr == 0) {
-                        dec_all[(kk & 1) * 128 + c] = __expf(gl);
-                        ega_s[c] = __expf(ga);
+                    if (tq == 0) {
+                        *reinterpret_cast<float2 *>(dec_all + (kk & 1) * 128 + c0) =
+                            make_float2(ex2_approx(kLog2e * glx), ex2_approx(kLog2e * gly));
+                        *reinterpret_cast<float2 *>(ega_s + c0) =
+                            make_float2(ex2_approx(kLog2e * gax), ex2_approx(kLog2e * gay));
                     }
                 }
                 fence_proxy_async_smem();
@@ -763,11 +866,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_fence_after();
                 if (t == 0) KDA_TRACE_POINT(m, 3);
                 {
-                    const int c = t & 127, hr = t >> 7;
+                    {
+                        const int cp = ((warp - 4) & 3) * 16 + (lane & 15);
+                        const int tq = 2 * ((warp - 4) >> 2) + (lane >> 4);
 #pragma unroll
-                    for (int rb = 0; rb < 4; ++rb)
-                        st_shared_v4(sbase + PR_KC + sw128(c, hr * 4 + rb), ktr[rb * 4], ktr[rb * 4 + 1],
-                                     ktr[rb * 4 + 2], ktr[rb * 4 + 3]);
+                        for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                            for (int h8 = 0; h8 < 2; ++h8) {
+                                const uint32_t *w4 = ktr + ch * 8 + h8 * 4;
+                                st_shared_v4(sbase + PR_KC + sw128(2 * cp + ch, 2 * tq + h8), w4[0], w4[1], w4[2],
+                                             w4[3]);
+                            }
+                    }
                     uint32_t a[32];
                     tmem_ld32(tmem + lane_base + COL_P1 + half * 32, a);
                     tmem_wait_ld();
@@ -827,18 +937,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (t < 128) {
                         const int wb = t >> 5, li = t & 31;
                         if (li < 16) {
+                            // column li of the inverse of diagonal block wb, row by row; the block's
+                            // rows of A are read as float4 (entries on and above the diagonal are 0)
                             float x[16];
 #pragma unroll
                             for (int rr = 0; rr < 16; ++rr) {
                                 const float *arow = A + (16 * wb + rr) * AKK_LD + 16 * wb;
                                 float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-                                for (int j = 0; j < rr; ++j) {
-                                    const float pr = arow[j] * x[j];
-                                    if ((j & 3) == 0) a0 += pr;
-                                    else if ((j & 3) == 1) a1 += pr;
-                                    else if ((j & 3) == 2) a2 += pr;
-                                    else a3 += pr;
+                                for (int j4 = 0; j4 < (rr + 3) / 4; ++j4) {
+                                    const float4 av = *reinterpret_cast<const float4 *>(arow + 4 * j4);
+                                    if (4 * j4 + 0 < rr) a0 = fmaf(av.x, x[4 * j4 + 0], a0);
+                                    if (4 * j4 + 1 < rr) a1 = fmaf(av.y, x[4 * j4 + 1], a1);
+                                    if (4 * j4 + 2 < rr) a2 = fmaf(av.z, x[4 * j4 + 2], a2);
+                                    if (4 * j4 + 3 < rr) a3 = fmaf(av.w, x[4 * j4 + 3], a3);
                                 }
                                 x[rr] = ((rr == li) ? 1.f : 0.f) - ((a0 + a1) + (a2 + a3));
                             }
@@ -855,11 +967,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const float *arow = A + (16 * I + rr) * AKK_LD + 16 * J;
                         float p0 = 0.f, p1 = 0.f;
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const float a = arow[j];
-                            const float2 tv = *reinterpret_cast<const float2 *>(T + (16 * J + j) * AKK_LD + 16 * J + cc);
-                            p0 = fmaf(a, tv.x, p0);
-                            p1 = fmaf(a, tv.y, p1);
+                        for (int j4 = 0; j4 < 4; ++j4) {
+                            const float4 av = *reinterpret_cast<const float4 *>(arow + 4 * j4);
+                            const float a4[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 tv =
+                                    *reinterpret_cast<const float2 *>(T + (16 * J + 4 * j4 + e) * AKK_LD + 16 * J + cc);
+                                p0 = fmaf(a4[e], tv.x, p0);
+                                p1 = fmaf(a4[e], tv.y, p1);
+                            }
                         }
                         *reinterpret_cast<float2 *>(P + blk * 256 + rr * 16 + cc) = make_float2(p0, p1);
                         named_bar_sync(2, 256);
@@ -867,42 +984,62 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         p0 = 0.f;
                         p1 = 0.f;
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const float a = trow[j];
-                            const float2 pv = *reinterpret_cast<const float2 *>(P + blk * 256 + j * 16 + cc);
-                            p0 = fmaf(a, pv.x, p0);
-                            p1 = fmaf(a, pv.y, p1);
+                        for (int j4 = 0; j4 < 4; ++j4) {
+                            const float4 tv4 = *reinterpret_cast<const float4 *>(trow + 4 * j4);
+                            const float t4[4] = {tv4.x, tv4.y, tv4.z, tv4.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 pv = *reinterpret_cast<const float2 *>(P + blk * 256 + (4 * j4 + e) * 16 + cc);
+                                p0 = fmaf(t4[e], pv.x, p0);
+                                p1 = fmaf(t4[e], pv.y, p1);
+                            }
                         }
                         *reinterpret_cast<float2 *>(T + (16 * I + rr) * AKK_LD + 16 * J + cc) = make_float2(-p0, -p1);
                     }
                     named_bar_sync(2, 256);
                     if (t == 0) KDA_TRACE_POINT(m, 11);
-                    // (c) rows 32..63, columns 0..31: P2 = A[32:, :32] T[:32, :32]; T = -T[32:, 32:] P2
+                    // (c) rows 32..63, columns 0..31: P2 = A[32:, :32] T[:32, :32]; T = -T[32:, 32:] P2.
+                    // Lane = row, warp = 4-column group, so the T and P2 reads are warp-uniform
+                    // (broadcast) and the zero block T[0:16, 16:32] is skipped by whole warps. P2 is
+                    // stored with its 16-byte groups XOR-swizzled by row to keep the stores conflict-free.
                     {
-                        const int rr = t >> 3, c4 = (t & 7) * 4;
+                        const int rr = t & 31, c4 = (t >> 5) * 4;
                         const float *arow = A + (32 + rr) * AKK_LD;
                         float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+                        const int j4lo = c4 >= 16 ? 4 : 0;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float a = arow[j];
-                            const float4 tv = *reinterpret_cast<const float4 *>(T + j * AKK_LD + c4);
-                            p0 = fmaf(a, tv.x, p0);
-                            p1 = fmaf(a, tv.y, p1);
-                            p2 = fmaf(a, tv.z, p2);
-                            p3 = fmaf(a, tv.w, p3);
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            if (j4 < j4lo) continue;
+                            const float4 av = *reinterpret_cast<const float4 *>(arow + 4 * j4);
+                            const float a4[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float4 tv = *reinterpret_cast<const float4 *>(T + (4 * j4 + e) * AKK_LD + c4);
+                                p0 = fmaf(a4[e], tv.x, p0);
+                                p1 = fmaf(a4[e], tv.y, p1);
+                                p2 = fmaf(a4[e], tv.z, p2);
+                                p3 = fmaf(a4[e], tv.w, p3);
+                            }
                         }
-                        *reinterpret_cast<float4 *>(P + rr * 32 + c4) = make_float4(p0, p1, p2, p3);
+                        *reinterpret_cast<float4 *>(P + rr * 32 + (((c4 >> 2) ^ (rr & 7)) << 2)) =
+                            make_float4(p0, p1, p2, p3);
                         named_bar_sync(2, 256);
                         const float *trow = T + (32 + rr) * AKK_LD + 32;
                         p0 = p1 = p2 = p3 = 0.f;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float a = trow[j];
-                            const float4 pv = *reinterpret_cast<const float4 *>(P + j * 32 + c4);
-                            p0 = fmaf(a, pv.x, p0);
-                            p1 = fmaf(a, pv.y, p1);
-                            p2 = fmaf(a, pv.z, p2);
-                            p3 = fmaf(a, pv.w, p3);
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 tv4 = *reinterpret_cast<const float4 *>(trow + 4 * j4);
+                            const float t4[4] = {tv4.x, tv4.y, tv4.z, tv4.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = 4 * j4 + e;
+                                const float4 pv =
+                                    *reinterpret_cast<const float4 *>(P + j * 32 + (((c4 >> 2) ^ (j & 7)) << 2));
+                                p0 = fmaf(t4[e], pv.x, p0);
+                                p1 = fmaf(t4[e], pv.y, p1);
+                                p2 = fmaf(t4[e], pv.z, p2);
+                                p3 = fmaf(t4[e], pv.w, p3);
+                            }
                         }
                         *reinterpret_cast<float4 *>(T + (32 + rr) * AKK_LD + c4) = make_float4(-p0, -p1, -p2, -p3);
                     }
@@ -930,7 +1067,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         }
                     }
                 }
+                if (t == 0) KDA_TRACE_POINT(m, 16);
                 fence_proxy_async_smem();
+                if (t == 0) KDA_TRACE_POINT(m, 17);
                 named_bar_sync(2, 256);
                 if (t == 0) {
                     mbar_arrive(BAR(PB_SOLVE_DONE));
@@ -1032,6 +1171,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     }
 
+    if (is_chain && tid == 128) {
+        KDA_TRACE_CLUSTER(1, globaltimer());
+        KDA_TRACE_CLUSTER(6, static_cast<unsigned long long>(clock64()));
+    }
     // ---------------------------------------------------------------- teardown
     if (*abort_flag) {
         // let any copy still in flight land before the CTA's memory is released
@@ -1191,6 +1334,12 @@ cudaError_t launch_fwd_tc_noalloc(const FwdParams &p, int64_t rows, cudaStream_t
 #ifdef KDA_TRACE
 extern "C" int kda_trace_read(unsigned long long *host) {
     return static_cast<int>(cudaMemcpyFromSymbol(host, g_kda_trace, sizeof(g_kda_trace)));
+}
+extern "C" int kda_trace_set_cluster(int c) {
+    return static_cast<int>(cudaMemcpyToSymbol(g_kda_trace_cluster, &c, sizeof(int)));
+}
+extern "C" int kda_trace_read_clusters(unsigned long long *host) {
+    return static_cast<int>(cudaMemcpyFromSymbol(host, g_kda_cluster_trace, sizeof(g_kda_cluster_trace)));
 }
 #endif
 
