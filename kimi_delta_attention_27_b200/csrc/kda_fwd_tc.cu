@@ -85,22 +85,28 @@ constexpr int C = kChunk;
 constexpr int NS = 4;          // CTAs per cluster: 1 chain + 3 prep
 constexpr int NPREP = NS - 1;
 constexpr int NTHREADS = 384;
-constexpr int NRING = 6;       // ring slots per cluster (multiple of NPREP)
+#ifndef KDA_NRING
+#define KDA_NRING 6
+#endif
+constexpr int NRING = KDA_NRING;  // ring slots per cluster (a multiple of NPREP)
+static_assert(NRING % 3 == 0 && NRING >= 6 && NRING <= 15, "ring depth");
 
-// ---- operand set of one chunk (same byte layout in the global ring and in smem)
-//   Kt^T fp16 [128 x 64] | -W^T bf16 [128 x 64] | Qt^T bf16 [128 x 64] |
-//   UV fp16 [128 x 128] as two 64-column blocks | e^Gl fp32 [128]
-constexpr uint32_t SET_KT = 0, SET_W = 16384, SET_Q = 32768, SET_UV = 49152, SET_DEC = 81920;
+// ---- operand set of one chunk (same byte layout in the global ring and in smem), 128B-swizzled tiles:
+//   Kt^T fp16 [128 key][64 token]              B operand of C3^T (K-major)
+//   -W^T, Qt^T bf16 [128 key][64 token] each   together the B operand of the state product (MN-major)
+//   V fp16 [64 token][128 value], two boxes    A operand of the value-side product (MN-major)
+//   [T'; Aqk T'] fp16 [128][64 token]          B operand of the value-side product (K-major)
+//   e^Gl fp32 [128]
+constexpr uint32_t SET_KT = 0, SET_W = 16384, SET_Q = 32768, SET_V = 49152, SET_AV = 65536, SET_DEC = 81920;
 constexpr uint32_t SET_BYTES = SET_DEC + 512;      // 82432
 constexpr uint32_t SET_STRIDE = 83968;             // 82 KB, 1024-aligned
 constexpr uint64_t RING_BYTES = static_cast<uint64_t>(NRING) * SET_STRIDE;
 constexpr int kMaxRings = 256;                     // indexed by the chain CTA's SM id
 
-// ---- chain CTA shared memory
+// ---- chain CTA shared memory: two operand-set slots (the output tile is staged over a
+// slot's V block once the value-side product has read it)
 constexpr uint32_t CH_SLOT = 0;                    // 2 x SET_STRIDE
-constexpr uint32_t CH_SP = 2 * SET_STRIDE;         // S' [128 x 128] bf16 MN-major SW128 (two 16 KB blocks)
-constexpr uint32_t CH_DL = CH_SP + 32768;          // D  [64 x 128] fp16 MN-major SW128 (two 8 KB blocks)
-constexpr uint32_t CH_MISC = CH_DL + 16384;
+constexpr uint32_t CH_MISC = 2 * SET_STRIDE;
 // ---- prep CTA shared memory
 constexpr uint32_t PR_STG = 0;                     // q 16 KB, k 16 KB, g 32 KB, v 16 KB
 constexpr uint32_t STG_Q = 0, STG_K = 16384, STG_G = 32768, STG_V = 65536, STAGE_TX = 65536, VSTAGE_TX = 16384;
@@ -115,7 +121,8 @@ constexpr uint32_t PR_AQB = PR_TB + 8192;          // Aqk bf16
 constexpr uint32_t PR_WP = PR_AQB + 8192;          // W'^T bf16
 constexpr uint32_t PR_MISC = PR_WP + 16384;
 static_assert(PR_P + 4096 <= PR_AVT, "prep map");
-static_assert(PR_AVT % 1024 == 0 && PR_WP % 1024 == 0 && CH_SP % 1024 == 0 && PR_KH % 1024 == 0, "alignment");
+static_assert(PR_AVT % 1024 == 0 && PR_WP % 1024 == 0 && PR_AKK % 1024 == 0 && PR_KH % 1024 == 0 &&
+                  SET_STRIDE % 1024 == 0 && SET_V % 1024 == 0, "alignment");
 
 // misc area (offsets from the misc base of either role)
 constexpr uint32_t M_BAR = 0;                      // up to 32 barriers
@@ -132,8 +139,8 @@ enum {
     CB_SFREE = 2,    // 2: smem slot consumed (8 epilogue warps, the output store warp, the release warp)
     CB_C1_FULL = 4, CB_C3_FULL = 8,
     CB_O_READY = 9,  // output tile staged in the slot (4 warps)
-    CB_READY = 10,   // 6: ring slot written by a prep CTA (remote arrival)
-    CB_COUNT = 16
+    CB_READY = 10,   // NRING: ring slot written by a prep CTA (remote arrival)
+    CB_COUNT = CB_READY + NRING
 };
 // prep barriers
 enum {
@@ -144,14 +151,15 @@ enum {
     PB_OUTC_READY,      // Qt^T (over the AV operand), UV (over A / T), e^Gl final
     PB_OUTAB_FREE,      // publisher has read parts A and B out
     PB_OUTC_FREE,       // publisher has read part C out
-    PB_RING_FREE = 15,  // 6: ring slot released by the chain CTA (remote arrival)
-    PB_COUNT = 21
+    PB_RING_FREE = 15,  // NRING: ring slot released by the chain CTA (remote arrival)
+    PB_COUNT = PB_RING_FREE + NRING
 };
 static_assert(CB_COUNT * 8 <= M_BETA && PB_COUNT * 8 <= M_BETA, "barrier area");
 
 // ---- TMEM columns
-constexpr uint32_t COL_C1 = 0, COL_C3 = 128;                                      // chain
-constexpr uint32_t COL_P1 = 0, COL_W = 64, COL_AV = 128, COL_Q = 192, COL_UV = 256;  // prep
+// chain: C1^T (two buffers), C3^T, S'^T (bf16 pairs), D^T (fp16 pairs)
+constexpr uint32_t COL_C1 = 0, COL_C3 = 256, COL_SP = 384, COL_DT = 448;
+constexpr uint32_t COL_P1 = 0, COL_W = 64, COL_AV = 128, COL_Q = 192;                 // prep
 constexpr uint32_t TMEM_COLS = 512;
 
 // ---- instruction descriptors (M = 128)
@@ -159,9 +167,9 @@ constexpr uint32_t ID_P1 = idesc_f16(128, 64, 1, 1, 1);      // bf16, A MN-major
 constexpr uint32_t ID_W = idesc_f16(128, 64, 1, 0, 0);       // bf16, K-major / K-major
 constexpr uint32_t ID_AV = idesc_f16(128, 64, 0, 0, 1);      // fp16, K-major / MN-major
 constexpr uint32_t ID_Q = idesc_f16(128, 64, 1, 0, 0);       // bf16
-constexpr uint32_t ID_UV = idesc_f16(128, 128, 0, 0, 1);     // fp16, A K-major, B MN-major
-constexpr uint32_t ID_STATE = idesc_f16(128, 128, 1, 1, 1);  // bf16, A MN-major, B MN-major
-constexpr uint32_t ID_C3 = idesc_f16(128, 128, 0, 0, 1);     // fp16
+constexpr uint32_t ID_UVT = idesc_f16(128, 128, 0, 1, 0);      // fp16, A (V) MN-major, B K-major
+constexpr uint32_t ID_STATE_T = idesc_f16(128, 128, 1, 0, 1);  // bf16, A (S'^T) in TMEM, B MN-major
+constexpr uint32_t ID_C3T = idesc_f16(128, 128, 0, 0, 0);      // fp16, A (D^T) in TMEM, B K-major
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 
@@ -219,6 +227,13 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
                  : "r"(addr)
                  : "memory");
     return v;
+}
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t x) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(x) : "memory");
+}
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+    __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return *reinterpret_cast<uint16_t *>(&h);
 }
 __device__ __forceinline__ void st_global_v4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
@@ -352,18 +367,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (is_chain) {
         // ======================================================================= chain CTA
         if (warp == 0) {
-            // ---- output tiles: staged in the slot's value-side rows 64..127 (two 64-column
-            // boxes, 128B swizzle); TMA-stored for full chunks, copied row by row otherwise
+            // ---- output tiles: staged over the slot's V block (two 64-channel boxes, 128B
+            // swizzle); TMA-stored for full chunks, copied row by row otherwise
             for (int n = 0; n < nch; ++n) {
                 const int sl = n & 1;
                 const int64_t t0 = bos + static_cast<int64_t>(n) * C;
                 const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
-                const uint32_t stage = sbase + CH_SLOT + sl * SET_STRIDE + SET_UV + 8192;
+                const uint32_t stage = sbase + CH_SLOT + sl * SET_STRIDE + SET_V;
                 if (!wait_bar(BAR(CB_O_READY), n & 1, abort_flag)) break;
                 if (L == C) {
                     if (lane == 0) {
                         tma_store_3d(&maps.o, stage, 0, h, static_cast<int32_t>(t0));
-                        tma_store_3d(&maps.o, stage + 16384, 64, h, static_cast<int32_t>(t0));
+                        tma_store_3d(&maps.o, stage + 8192, 64, h, static_cast<int32_t>(t0));
                         bulk_commit();
                         bulk_wait_read0();
                     }
@@ -371,7 +386,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     // partial chunk: rows < L only, 16 bytes per lane, a row is 2 x 8 chunks
                     for (int e = lane; e < L * 16; e += 32) {
                         const int rr = e >> 4, hb = (e >> 3) & 1, j = e & 7;
-                        const uint4 v = ld_shared_v4(stage + hb * 16384 + sw128(rr, j));
+                        const uint4 v = ld_shared_v4(stage + hb * 8192 + sw128(rr, j));
                         st_global_v4(p.out + ((t0 + rr) * H + h) * D + hb * 64 + j * 8, v.x, v.y, v.z, v.w);
                     }
                 }
@@ -413,192 +428,188 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 __syncwarp();
             }
         } else if (warp >= 4) {
-            // ---- epilogues: 8 warps; a warp covers TMEM lanes 32*(warp%4).. and value columns 64*half..
+            // ---- epilogues: 8 warps. The state is kept transposed: a thread owns S^T[v][j] for
+            // one value channel v = TMEM lane 32*(warp%4) + lane and 64 key channels
+            // j in [64*half, 64*half + 64). Per chunk (all products accumulate in fp32 TMEM):
+            //   C1^T = V^T [T'; Aqk T']^T + S'^T [-W; Qt]^T   columns 0..63: D^T, 64..127: O^T / scale
+            //   C3^T = D^T Kt                                  S^T <- e^Gl (.) S^T + C3^T
+            // The bf16 state copy S'^T and the fp16 pseudo-values D^T are written straight into
+            // TMEM, where they are the A operands of the next products.
             const int q4 = warp & 3, half = (warp - 4) >> 2;
-            const int row = q4 * 32 + lane;            // TMEM lane = state row k / chunk row
+            const int v = q4 * 32 + lane;              // value channel = TMEM lane
             const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
-            const int c0 = half * 64;                  // first value column of this thread
+            const int j0 = half * 64;                  // first key channel of this thread
             float S[64];
             if (p.h0) {
-                const size_t off = state_base + static_cast<size_t>(row) * D + c0;
                 if (p.h0_fp32) {
-                    const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(p.h0) + off);
+                    const float *src = static_cast<const float *>(p.h0) + state_base + v;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float4 x = src[j];
-                        S[4 * j] = x.x; S[4 * j + 1] = x.y; S[4 * j + 2] = x.z; S[4 * j + 3] = x.w;
-                    }
+                    for (int i = 0; i < 64; ++i) S[i] = src[static_cast<size_t>(j0 + i) * D];
                 } else {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.h0) + off);
+                    const uint16_t *src = static_cast<const uint16_t *>(p.h0) + state_base + v;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint4 x = src[j];
-                        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            S[8 * j + 2 * e] = lo_bf(w[e]);
-                            S[8 * j + 2 * e + 1] = hi_bf(w[e]);
-                        }
-                    }
+                    for (int i = 0; i < 64; ++i) S[i] = bf2f(src[static_cast<size_t>(j0 + i) * D]);
                 }
             } else {
 #pragma unroll
-                for (int j = 0; j < 64; ++j) S[j] = 0.f;
+                for (int i = 0; i < 64; ++i) S[i] = 0.f;
             }
-            // S' (bf16, MN-major: column block `half`, row `row`)
+            // S'^T (bf16, two key channels per TMEM column) -> columns COL_SP + 32*half
             auto write_sprime = [&]() {
-                const uint32_t base = sbase + CH_SP + half * 16384;
+                uint32_t w[32];
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    st_shared_v4(base + sw128(row, j), pack_bf16(S[8 * j], S[8 * j + 1]),
-                                 pack_bf16(S[8 * j + 2], S[8 * j + 3]), pack_bf16(S[8 * j + 4], S[8 * j + 5]),
-                                 pack_bf16(S[8 * j + 6], S[8 * j + 7]));
+                for (int i = 0; i < 32; ++i) w[i] = pack_bf16(S[2 * i], S[2 * i + 1]);
+                tmem_st32(tmem + lane_base + COL_SP + 32 * half, w);
+                tmem_wait_st();
             };
-            // The MMAs are issued by one thread of the epilogue warps as soon as their operands
-            // are in place (a named barrier among the writers), with no hop through another warp:
-            //   C1 = [-W; Qt] S'   (bf16; S' written by all 8 warps)
-            //   C3 = Kt^T D        (fp16; D written by the 4 warps of rows 0..63)
-            auto issue_c1 = [&](int n) -> bool {
+            // The products are issued by one thread (tid 128, a D^T warp) as soon as their operands
+            // are in place (a named barrier among the writers), with no hop through another warp.
+            // value-side product of chunk n into its C1^T buffer (no state involved); C1^T has two
+            // buffers, so chunk n's buffer was last read in chunk n - 2
+            auto issue_uv = [&](int n) -> bool {
                 const int s1 = n & 1;
                 const uint32_t slot = sbase + CH_SLOT + s1 * SET_STRIDE;
                 if (!wait_bar(BAR(CB_FULL + s1), (n >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tmem + COL_C1 + s1 * 128, smem_desc(slot + SET_V + ks * 2048, 8192, 1024, kSwizzle128),
+                            smem_desc(slot + SET_AV + ks * 32, 16, 1024, kSwizzle128), ID_UVT, ks > 0);
+                return true;
+            };
+            auto issue_state = [&](int n) {
+                const int s1 = n & 1;
+                const uint32_t slot = sbase + CH_SLOT + s1 * SET_STRIDE;
+                tc_fence_after();
                 KDA_TRACE_POINT(n, 13);
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_f16(tmem + COL_C1, smem_desc(slot + SET_W + ks * 2048, 16384, 1024, kSwizzle128),
-                            smem_desc(sbase + CH_SP + ks * 2048, 16384, 1024, kSwizzle128), ID_STATE, ks > 0);
+                    mma_f16_ts(tmem + COL_C1 + s1 * 128, tmem + COL_SP + ks * 8,
+                               smem_desc(slot + SET_W + ks * 2048, 16384, 1024, kSwizzle128), ID_STATE_T, 1);
                 mma_commit(BAR(CB_C1_FULL));
                 KDA_TRACE_POINT(n, 3);
-                return true;
             };
             auto issue_c3 = [&](int n) {
                 const uint32_t slot = sbase + CH_SLOT + (n & 1) * SET_STRIDE;
                 tc_fence_after();
                 KDA_TRACE_POINT(n, 4);
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tmem + COL_C3, smem_desc(slot + SET_KT + ks * 32, 16, 1024, kSwizzle128),
-                            smem_desc(sbase + CH_DL + ks * 2048, 8192, 1024, kSwizzle128), ID_C3, ks > 0);
+                    mma_f16_ts(tmem + COL_C3, tmem + COL_DT + ks * 8,
+                               smem_desc(slot + SET_KT + ks * 32, 16, 1024, kSwizzle128), ID_C3T, ks > 0);
                 mma_commit(BAR(CB_C3_FULL));
                 KDA_TRACE_POINT(n, 5);
             };
             write_sprime();
-            fence_proxy_async_smem();
             tc_fence_before();
             named_bar_sync(4, 256);
-            if (tid == 128 && nch > 0) issue_c1(0);
+            if (tid == 128 && nch > 0) {
+                if (issue_uv(0)) issue_state(0);
+            }
             __syncwarp();
             for (int n = 0; n < nch; ++n) {
                 const int sl = n & 1;
-                const int64_t t0 = bos + static_cast<int64_t>(n) * C;
-                const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
                 if (!wait_bar(BAR(CB_C1_FULL), n & 1, abort_flag)) break;
                 tc_fence_after();
                 if (tid == 128) KDA_TRACE_POINT(n, 9);
-                {
-                    // value side of this row (U for rows < 64, Aqk U below), fp16; the row's 64
-                    // columns are done as two halves so that the TMEM and shared-memory loads of a
-                    // half are in flight together
-                    const uint32_t uvb = sbase + CH_SLOT + sl * SET_STRIDE + SET_UV + half * 16384;
+                const uint32_t acc = tmem + lane_base + COL_C1 + sl * 128 + 64 * half;
+                bool ok = true;
+                if (half == 0) {
+                    // pseudo-values D^T[v][t] -> fp16, two tokens per TMEM column (A operand of C3^T)
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(acc, r0);
+                    tmem_ld32(acc + 32, r1);
+                    tmem_wait_ld();
+                    if (tid == 128) KDA_TRACE_POINT(n, 0);
+                    uint32_t w[32];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) w[i] = pack_f16(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        w[16 + i] = pack_f16(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
+                    tmem_st32(tmem + lane_base + COL_DT, w);
+                    tmem_wait_st();
+                    if (tid == 128) KDA_TRACE_POINT(n, 1);
+                    tc_fence_before();
+                    named_bar_sync(3, 128);
+                    if (tid == 128) {
+                        issue_c3(n);
+                        // the next chunk's value-side product follows C3^T on the tensor pipe; this
+                        // thread waits for its slot here, so that the product runs during the C3^T
+                        // epilogue rather than ahead of the next state product
+                        if (n + 1 < nch) ok = issue_uv(n + 1);
+                    }
+                    __syncwarp();
+                } else {
+                    // output tile O[t][v] = scale * C1^T[v][64 + t] (bf16), staged over the slot's V
+                    // block (two 64-channel boxes, 128B swizzle) for the store warp
+                    const uint32_t stage = sbase + CH_SLOT + sl * SET_STRIDE + SET_V + (v >> 6) * 8192;
+                    const uint32_t vc = static_cast<uint32_t>(v & 63);
+                    const float sc = p.scale;
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         uint32_t r[32];
-                        tmem_ld32(tmem + lane_base + COL_C1 + c0 + 32 * hh, r);
-                        uint4 u4[4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) u4[j] = ld_shared_v4(uvb + sw128(row, 4 * hh + j));
+                        tmem_ld32(acc + 32 * hh, r);
                         tmem_wait_ld();
-                        if (tid == 128 && hh == 0) KDA_TRACE_POINT(n, 0);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint32_t uw[4] = {u4[j].x, u4[j].y, u4[j].z, u4[j].w};
-                            const uint32_t *rr = r + 8 * j;
-                            float x[8];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 uf = __half22float2(*reinterpret_cast<const __half2 *>(&uw[e]));
-                                x[2 * e] = __uint_as_float(rr[2 * e]) + uf.x;
-                                x[2 * e + 1] = __uint_as_float(rr[2 * e + 1]) + uf.y;
-                            }
-                            const int jj = 4 * hh + j;
-                            if (row < 64) {
-                                // pseudo-values D -> fp16 B operand of the state increment
-                                st_shared_v4(sbase + CH_DL + half * 8192 + sw128(row, jj), pack_f16(x[0], x[1]),
-                                             pack_f16(x[2], x[3]), pack_f16(x[4], x[5]), pack_f16(x[6], x[7]));
-                            } else {
-                                // output row -> staging tile over the value-side rows just consumed
-                                // (same bytes this thread read above); the store warp writes it out
-                                const float sc = p.scale;
-                                st_shared_v4(uvb + sw128(row, jj), pack_bf16(sc * x[0], sc * x[1]),
-                                             pack_bf16(sc * x[2], sc * x[3]), pack_bf16(sc * x[4], sc * x[5]),
-                                             pack_bf16(sc * x[6], sc * x[7]));
-                            }
+                        for (int i = 0; i < 32; ++i) {
+                            const uint32_t t = static_cast<uint32_t>(32 * hh + i);
+                            const uint32_t a = stage + t * 128u + ((((vc >> 3) ^ (t & 7u))) << 4) + (vc & 7u) * 2u;
+                            st_shared_u16(a, bf16_bits(sc * __uint_as_float(r[i])));
                         }
                     }
-                    if (tid == 128) KDA_TRACE_POINT(n, 1);
                     fence_proxy_async_smem();
-                    if (tid == 128) KDA_TRACE_POINT(n, 2);
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (tid == 128) KDA_TRACE_POINT(n, 6);
-                if (row < 64) {
-                    named_bar_sync(3, 128);
-                    if (tid == 128) issue_c3(n);
+                    tc_fence_before();
                     __syncwarp();
-                } else if (lane == 0) {
-                    mbar_arrive(BAR(CB_O_READY));
+                    if (lane == 0) mbar_arrive(BAR(CB_O_READY));
                 }
+                if (tid == 128) KDA_TRACE_POINT(n, 6);
+                if (!ok) break;
                 if (!wait_bar(BAR(CB_C3_FULL), n & 1, abort_flag)) break;
                 tc_fence_after();
                 if (tid == 128) KDA_TRACE_POINT(n, 10);
-                if (lane == 0) KDA_TRACE_POINT(n, 24 + warp - 4);
                 {
                     uint32_t r0[32], r1[32];
-                    tmem_ld32(tmem + lane_base + COL_C3 + c0, r0);
-                    tmem_ld32(tmem + lane_base + COL_C3 + c0 + 32, r1);
+                    tmem_ld32(tmem + lane_base + COL_C3 + j0, r0);
+                    tmem_ld32(tmem + lane_base + COL_C3 + j0 + 32, r1);
+                    const float *decp = reinterpret_cast<const float *>(sgen + CH_SLOT + sl * SET_STRIDE + SET_DEC) + j0;
                     tmem_wait_ld();
-                    const float dec =
-                        reinterpret_cast<const float *>(sgen + CH_SLOT + sl * SET_STRIDE + SET_DEC)[row];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) S[j] = fmaf(dec, S[j], __uint_as_float(r0[j]));
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 d4 = reinterpret_cast<const float4 *>(decp)[i4];
+                        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) S[32 + j] = fmaf(dec, S[32 + j], __uint_as_float(r1[j]));
+                        for (int e = 0; e < 4; ++e) S[4 * i4 + e] = fmaf(dv[e], S[4 * i4 + e], __uint_as_float(r0[4 * i4 + e]));
+                    }
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 d4 = reinterpret_cast<const float4 *>(decp)[8 + i4];
+                        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            S[32 + 4 * i4 + e] = fmaf(dv[e], S[32 + 4 * i4 + e], __uint_as_float(r1[4 * i4 + e]));
+                    }
                 }
                 if (tid == 128) KDA_TRACE_POINT(n, 8);
-                if (n + 1 < nch) {
-                    write_sprime();
-                    if (tid == 128) KDA_TRACE_POINT(n, 7);
-                    fence_proxy_async_smem();
-                    if (tid == 128) KDA_TRACE_POINT(n, 14);
-                }
+                if (n + 1 < nch) write_sprime();
+                if (tid == 128) KDA_TRACE_POINT(n, 7);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(BAR(CB_SFREE + sl));
                 if (n + 1 < nch) {
                     named_bar_sync(4, 256);
-                    bool ok = true;
-                    if (tid == 128) ok = issue_c1(n + 1);
+                    if (tid == 128) issue_state(n + 1);
                     __syncwarp();
-                    if (!ok) break;
                 }
                 if (tid == 128) KDA_TRACE_POINT(n, 11);
-                if (lane == 0) KDA_TRACE_POINT(n, 16 + warp - 4);
             }
-            // final state
+            // final state: hT[j][v], coalesced across the warp for each key channel j
             if (p.hT && !*abort_flag) {
-                const size_t off = state_base + static_cast<size_t>(row) * D + c0;
                 if (p.hT_fp32) {
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.hT) + off);
+                    float *dst = static_cast<float *>(p.hT) + state_base + v;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+                    for (int i = 0; i < 64; ++i) dst[static_cast<size_t>(j0 + i) * D] = S[i];
                 } else {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.hT) + off);
+                    uint16_t *dst = static_cast<uint16_t *>(p.hT) + state_base + v;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        dst[j] = make_uint4(pack_bf16(S[8 * j], S[8 * j + 1]), pack_bf16(S[8 * j + 2], S[8 * j + 3]),
-                                            pack_bf16(S[8 * j + 4], S[8 * j + 5]),
-                                            pack_bf16(S[8 * j + 6], S[8 * j + 7]));
+                    for (int i = 0; i < 64; ++i) dst[static_cast<size_t>(j0 + i) * D] = bf16_bits(S[i]);
                 }
             }
         }
@@ -661,11 +672,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int ks = 0; ks < 4; ++ks)
                         mma_f16(tmem + COL_Q, smem_desc(sbase + PR_WP + ks * 32, 16, 1024, kSwizzle128),
                                 smem_desc(sbase + PR_AQB + ks * 32, 16, 1024, kSwizzle128), ID_Q, ks > 0);
-                    // [T'; Aqk T'] V = [U; Aqk U]  (fp16, N = 128)
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tmem + COL_UV, smem_desc(sbase + PR_AVT + ks * 32, 16, 1024, kSwizzle128),
-                                smem_desc(sbase + PR_STG + STG_V + ks * 2048, 8192, 1024, kSwizzle128), ID_UV,
-                                ks > 0);
                     mma_commit(BAR(PB_Q_DONE));
                 }
                 __syncwarp();
@@ -700,13 +706,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!wait_bar(BAR(PB_OUTC_READY), kk & 1, abort_flag)) break;
                 if (lane == 0) {
                     KDA_TRACE_POINT(m, 22);
-                    bulk_s2g(set + SET_Q, sbase + PR_AVT, 16384);
-                    bulk_s2g(set + SET_UV, sbase + PR_AKK, 32768);
+                    bulk_s2g(set + SET_Q, sbase + PR_AKK, 16384);
+                    bulk_s2g(set + SET_V, sbase + PR_STG + STG_V, 16384);
+                    bulk_s2g(set + SET_AV, sbase + PR_AVT, 16384);
                     bulk_s2g(set + SET_DEC, misc + M_DEC + (kk & 1) * 512, 512);
                     bulk_commit();
                     bulk_wait_read0();
                     KDA_TRACE_POINT(m, 23);
                     mbar_arrive(BAR(PB_OUTC_FREE));
+                    mbar_arrive(BAR(PB_VSTAGE_FREE));
                     bulk_wait0();
                     KDA_TRACE_POINT(m, 24);
                     fence_proxy_async_global();
@@ -1121,7 +1129,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     KDA_TRACE_POINT(m, 6);
                 }
 
-                // -------- Qt = (Qh - Aqk W') e^Ga (over the AV operand) and UV (over A / T)
+                // -------- Qt = (Qh - Aqk W') e^Ga, over the dead A workspace (the value side of the
+                // chunk is computed by the chain CTA from V and [T'; Aqk T'])
                 if (!wait_bar(BAR(PB_Q_DONE), kk & 1, abort_flag)) break;
                 tc_fence_after();
                 if (t == 0) KDA_TRACE_POINT(m, 7);
@@ -1140,33 +1149,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         for (int e = 0; e < 4; ++e)
                             o[e] = pack_bf16(sc * (lo_bf(qw[e]) - __uint_as_float(a[8 * j + 2 * e])),
                                              sc * (hi_bf(qw[e]) - __uint_as_float(a[8 * j + 2 * e + 1])));
-                        st_shared_v4(sbase + PR_AVT + sw128(lrow, jj), o[0], o[1], o[2], o[3]);
+                        st_shared_v4(sbase + PR_AKK + sw128(lrow, jj), o[0], o[1], o[2], o[3]);
                     }
                     if (t == 0) KDA_TRACE_POINT(m, 14);
-                    // value side UV = [U; Aqk U], row lrow, 64 columns of block `half`
-                    uint32_t u0[32], u1[32];
-                    tmem_ld32(tmem + lane_base + COL_UV + half * 64, u0);
-                    tmem_ld32(tmem + lane_base + COL_UV + half * 64 + 32, u1);
-                    tmem_wait_ld();
-                    const uint32_t uvb = sbase + PR_AKK + half * 16384;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint32_t *x = j < 4 ? u0 + 8 * j : u1 + 8 * (j - 4);
-                        st_shared_v4(uvb + sw128(lrow, j), pack_f16(__uint_as_float(x[0]), __uint_as_float(x[1])),
-                                     pack_f16(__uint_as_float(x[2]), __uint_as_float(x[3])),
-                                     pack_f16(__uint_as_float(x[4]), __uint_as_float(x[5])),
-                                     pack_f16(__uint_as_float(x[6]), __uint_as_float(x[7])));
-                    }
                 }
                 if (t == 0) KDA_TRACE_POINT(m, 15);
                 // hand the finished set to the publisher
                 fence_proxy_async_smem();
                 tc_fence_before();
                 named_bar_sync(2, 256);
-                if (t == 0) {
-                    mbar_arrive(BAR(PB_VSTAGE_FREE));
-                    mbar_arrive(BAR(PB_OUTC_READY));
-                }
+                if (t == 0) mbar_arrive(BAR(PB_OUTC_READY));
             }
         }
     }
