@@ -637,45 +637,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 __syncwarp();
             }
-        } else if (warp == 1) {
-            // ---- prep MMA issuer
-            int kk = 0;
-            for (int m = first; m < nch; m += NPREP, ++kk) {
-                if (!wait_bar(BAR(PB_EW_DONE), kk & 1, abort_flag)) break;
-                tc_fence_after();
-                if (lane == 0) {
-                    // [Kh; Qh] Kc^T : A = Kh^T | Qh^T (MN-major, 64-row blocks 16 KB apart), B = Kc^T
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_f16(tmem + COL_P1, smem_desc(sbase + PR_KH + ks * 2048, 16384, 1024, kSwizzle128),
-                                smem_desc(sbase + PR_KC + ks * 2048, 16384, 1024, kSwizzle128), ID_P1, ks > 0);
-                    mma_commit(BAR(PB_P1_DONE));
-                }
-                __syncwarp();
-                if (!wait_bar(BAR(PB_SOLVE_DONE), kk & 1, abort_flag)) break;
-                tc_fence_after();
-                if (lane == 0) {
-                    // W'^T = Kh^T T'^T (bf16)
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tmem + COL_W, smem_desc(sbase + PR_KH + ks * 32, 16, 1024, kSwizzle128),
-                                smem_desc(sbase + PR_TB + ks * 32, 16, 1024, kSwizzle128), ID_W, ks > 0);
-                    // [T'; Aqk] T' (fp16); rows 64..127 (Aqk T') are used
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tmem + COL_AV, smem_desc(sbase + PR_AVT + ks * 32, 16, 1024, kSwizzle128),
-                                smem_desc(sbase + PR_AVT + ks * 2048, 16384, 1024, kSwizzle128), ID_AV, ks > 0);
-                    mma_commit(BAR(PB_WAV_DONE));
-                }
-                __syncwarp();
-                if (!wait_bar(BAR(PB_WEPI_DONE), kk & 1, abort_flag)) break;
-                tc_fence_after();
-                if (lane == 0) {
-                    // W'^T Aqk^T (bf16)
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tmem + COL_Q, smem_desc(sbase + PR_WP + ks * 32, 16, 1024, kSwizzle128),
-                                smem_desc(sbase + PR_AQB + ks * 32, 16, 1024, kSwizzle128), ID_Q, ks > 0);
-                    mma_commit(BAR(PB_Q_DONE));
-                }
-                __syncwarp();
-            }
         } else if (warp == 3) {
             // ---- publisher: finished parts of the operand set (smem) -> ring slot (global),
             // each by bulk stores as soon as the part is final
@@ -851,9 +812,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 fence_proxy_async_smem();
                 named_bar_sync(2, 256);
+                // The prep MMAs are issued by this thread right after the barrier that ends the
+                // phase writing their operands (no hop through another warp).
                 if (t == 0) {
-                    mbar_arrive(BAR(PB_EW_DONE));
                     mbar_arrive(BAR(PB_STAGE_FREE));
+                    tc_fence_after();
+                    // [Kh; Qh] Kc^T : A = Kh^T | Qh^T (MN-major, 64-row blocks 16 KB apart), B = Kc^T
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_f16(tmem + COL_P1, smem_desc(sbase + PR_KH + ks * 2048, 16384, 1024, kSwizzle128),
+                                smem_desc(sbase + PR_KC + ks * 2048, 16384, 1024, kSwizzle128), ID_P1, ks > 0);
+                    mma_commit(BAR(PB_P1_DONE));
                     KDA_TRACE_POINT(m, 2);
                 }
                 // value tile bf16 -> fp16 in place (B operand of the value-side MMA)
@@ -1080,7 +1048,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (t == 0) KDA_TRACE_POINT(m, 17);
                 named_bar_sync(2, 256);
                 if (t == 0) {
-                    mbar_arrive(BAR(PB_SOLVE_DONE));
+                    tc_fence_after();
+                    // W'^T = Kh^T T'^T (bf16)
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(tmem + COL_W, smem_desc(sbase + PR_KH + ks * 32, 16, 1024, kSwizzle128),
+                                smem_desc(sbase + PR_TB + ks * 32, 16, 1024, kSwizzle128), ID_W, ks > 0);
+                    // [T'; Aqk] T' (fp16); rows 64..127 (Aqk T') are used
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(tmem + COL_AV, smem_desc(sbase + PR_AVT + ks * 32, 16, 1024, kSwizzle128),
+                                smem_desc(sbase + PR_AVT + ks * 2048, 16384, 1024, kSwizzle128), ID_AV, ks > 0);
+                    mma_commit(BAR(PB_WAV_DONE));
                     KDA_TRACE_POINT(m, 4);
                 }
 
@@ -1124,8 +1101,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_fence_before();
                 named_bar_sync(2, 256);
                 if (t == 0) {
-                    mbar_arrive(BAR(PB_WEPI_DONE));
                     mbar_arrive(BAR(PB_OUTB_READY));
+                    tc_fence_after();
+                    // W'^T Aqk^T (bf16)
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(tmem + COL_Q, smem_desc(sbase + PR_WP + ks * 32, 16, 1024, kSwizzle128),
+                                smem_desc(sbase + PR_AQB + ks * 32, 16, 1024, kSwizzle128), ID_Q, ks > 0);
+                    mma_commit(BAR(PB_Q_DONE));
                     KDA_TRACE_POINT(m, 6);
                 }
 
