@@ -10,20 +10,18 @@
 //   [Akk_raw; Aqk] = [Kh; Qh] Kc^T                          (S2, one M=128 MMA)
 //   Akk = strict_lower(diag(beta) Akk_raw), Aqk = lower(Aqk)
 //   T' = (I + Akk)^-1 diag(beta)                            (S3, blocked substitution)
-//   W' = T' Kh;  W = W' diag(e^Ga)                          (S4)
-//   Qt = (Qh - Aqk W') diag(e^Ga)                           (read-out folded with the
-//                                                            intra-chunk attention)
-//   UV = [T'; Aqk T'] V = [U; Aqk U]                        (S4, value side)
-//   X  = [-W; Qt] S + UV      ->  X[0:64] = D (pseudo-values), X[64:128] = O / scale (S5+S6)
+//   W' = T' Kh;  W = W' diag(e^Ga);  U = T' V               (S4)
+//   Qd = Qh diag(e^Ga) = Q e^G                              (decayed queries)
+//   D  = U - W S                                            (S5, pseudo-values)
+//   O  = scale (Qd S + Aqk D)                               (S6, inter + intra chunk)
 //   S <- diag(e^Gl) S + Kt^T D                              (S7)
 //
 // Work split: one 4-CTA cluster per (sequence, head).
 //  * rank 0 ("chain") owns the whole fp32 state (128 x 128) and runs the sequential
-//    part, S5-S7, with 128-column MMAs: the dependent-step latency of a tcgen05 MMA
-//    is the same for N = 32 and N = 128, so the state is not split.
+//    part, S5-S7 (and U = T' V), with 128-column MMAs: the dependent-step latency of a
+//    tcgen05 MMA barely depends on N up to 128, so the state is not split.
 //  * ranks 1-3 ("prep") each prepare every third chunk (S0-S4: gates, decayed
-//    blocks, UT solve, W / Qt / Kt and the value side UV), writing the finished
-//    80.5 KB operand set
+//    blocks, UT solve, W, Qd, Kt), writing the finished 80.5 KB operand set
 //    into a per-cluster ring of 6 slots in global memory (it stays in L2); the
 //    chain CTA pulls each set with one TMA bulk load. Shared memory of another
 //    CTA (DSMEM) carries only barrier signals: its bulk bandwidth is a fraction
@@ -31,10 +29,10 @@
 //  Every input byte is read from HBM once (q, k, v, g, beta by a prep CTA) and
 //  every output byte written once (by the chain CTA).
 //
-// Precision: anchored factors (Kh, Qh, Kc), W, Qt and the state copy S' are bf16;
-// T', Aqk T', V, UV, Kt and D are fp16 (10-bit mantissa) because the state update is
-// most sensitive to them; every product accumulates in fp32 (TMEM) and the state itself
-// is carried in fp32 registers.
+// Precision: anchored factors (Kh, Qh, Kc), W, Qd and the state copy S' are bf16;
+// T', Aqk, V, Kt and D are fp16 (10-bit mantissa) because the state update is most
+// sensitive to them; every product accumulates in fp32 (TMEM) and the state itself is
+// carried in fp32 registers.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -93,20 +91,23 @@ static_assert(NRING % 3 == 0 && NRING >= 6 && NRING <= 15, "ring depth");
 
 // ---- operand set of one chunk (same byte layout in the global ring and in smem), 128B-swizzled tiles:
 //   Kt^T fp16 [128 key][64 token]              B operand of C3^T (K-major)
-//   -W^T, Qt^T bf16 [128 key][64 token] each   together the B operand of the state product (MN-major)
+//   -W^T, Qd^T bf16 [128 key][64 token] each   together the B operand of the state product (MN-major)
 //   V fp16 [64 token][128 value], two boxes    A operand of the value-side product (MN-major)
-//   [T'; Aqk T'] fp16 [128][64 token]          B operand of the value-side product (K-major)
+//   T' fp16 [64][64 token]                     B operand of the value-side product (K-major)
+//   Aqk fp16 [64 token][64 token]              B operand of the intra-chunk output product (K-major)
 //   e^Gl fp32 [128]
-constexpr uint32_t SET_KT = 0, SET_W = 16384, SET_Q = 32768, SET_V = 49152, SET_AV = 65536, SET_DEC = 81920;
-constexpr uint32_t SET_BYTES = SET_DEC + 512;      // 82432
+constexpr uint32_t SET_KT = 0, SET_W = 16384, SET_Q = 32768, SET_V = 49152, SET_T = 65536, SET_AQK = 73728,
+                   SET_DEC = 81920;
+constexpr uint32_t SET_TX = 4 * 16384 + 2 * 8192 + 512;   // bytes per set
 constexpr uint32_t SET_STRIDE = 83968;             // 82 KB, 1024-aligned
+static_assert(SET_DEC + 512 <= SET_STRIDE, "operand set");
 constexpr uint64_t RING_BYTES = static_cast<uint64_t>(NRING) * SET_STRIDE;
 constexpr int kMaxRings = 256;                     // indexed by the chain CTA's SM id
 
-// ---- chain CTA shared memory: two operand-set slots (the output tile is staged over a
-// slot's V block once the value-side product has read it)
+// ---- chain CTA shared memory: two operand-set slots and two output staging tiles
 constexpr uint32_t CH_SLOT = 0;                    // 2 x SET_STRIDE
-constexpr uint32_t CH_MISC = 2 * SET_STRIDE;
+constexpr uint32_t CH_OST = 2 * SET_STRIDE;        // 2 x [64 token][128 value] bf16 (two 64-channel boxes)
+constexpr uint32_t CH_MISC = CH_OST + 2 * 16384;
 // ---- prep CTA shared memory
 constexpr uint32_t PR_STG = 0;                     // q 16 KB, k 16 KB, g 32 KB, v 16 KB
 constexpr uint32_t STG_Q = 0, STG_K = 16384, STG_G = 32768, STG_V = 65536, STAGE_TX = 65536, VSTAGE_TX = 16384;
@@ -115,13 +116,11 @@ constexpr uint32_t AKK_LD = 68;                    // fp32 row stride of A and T
 constexpr uint32_t PR_AKK = PR_KC + 16384;         // 17408 B
 constexpr uint32_t PR_T = PR_AKK + 17408;          // 17408 B
 constexpr uint32_t PR_P = PR_T + 17408;            // 4096 B
-constexpr uint32_t PR_AVT = 169984;                // [T'h; (Aqk T')_h] fp16, 128 rows K-major SW128
+constexpr uint32_t PR_AVT = 169984;                // [T'; Aqk] fp16, 128 rows K-major SW128
 constexpr uint32_t PR_TB = PR_AVT + 16384;         // T' bf16
-constexpr uint32_t PR_AQB = PR_TB + 8192;          // Aqk bf16
-constexpr uint32_t PR_WP = PR_AQB + 8192;          // W'^T bf16
-constexpr uint32_t PR_MISC = PR_WP + 16384;
+constexpr uint32_t PR_MISC = PR_TB + 8192;
 static_assert(PR_P + 4096 <= PR_AVT, "prep map");
-static_assert(PR_AVT % 1024 == 0 && PR_WP % 1024 == 0 && PR_AKK % 1024 == 0 && PR_KH % 1024 == 0 &&
+static_assert(PR_AVT % 1024 == 0 && PR_AKK % 1024 == 0 && PR_KH % 1024 == 0 &&
                   SET_STRIDE % 1024 == 0 && SET_V % 1024 == 0, "alignment");
 
 // misc area (offsets from the misc base of either role)
@@ -136,9 +135,12 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 // chain barriers
 enum {
     CB_FULL = 0,     // 2: operand set landed in smem slot (1 arrival + tx)
-    CB_SFREE = 2,    // 2: smem slot consumed (8 epilogue warps, the output store warp, the release warp)
-    CB_C1_FULL = 4, CB_C3_FULL = 8,
-    CB_O_READY = 9,  // output tile staged in the slot (4 warps)
+    CB_SFREE = 2,    // 2: smem slot consumed (8 epilogue warps, the release warp, the output-product warp)
+    CB_C1_FULL = 4,  // value-side + state products done
+    CB_O_FULL = 5,   // intra-chunk output product done
+    CB_OST_FREE = 6, // 2: output staging tile read out by the store warp
+    CB_C3_FULL = 8,
+    CB_O_READY = 9,  // output tile staged (4 warps)
     CB_READY = 10,   // NRING: ring slot written by a prep CTA (remote arrival)
     CB_COUNT = CB_READY + NRING
 };
@@ -148,7 +150,7 @@ enum {
     PB_WAV_DONE, PB_WEPI_DONE, PB_Q_DONE,
     PB_OUTA_READY,      // Kt^T final (over Kc^T)
     PB_OUTB_READY,      // -W^T final (over Kh^T)
-    PB_OUTC_READY,      // Qt^T (over the AV operand), UV (over A / T), e^Gl final
+    PB_OUTC_READY,      // Qd^T (over A), T' and Aqk, V, e^Gl final
     PB_OUTAB_FREE,      // publisher has read parts A and B out
     PB_OUTC_FREE,       // publisher has read part C out
     PB_RING_FREE = 15,  // NRING: ring slot released by the chain CTA (remote arrival)
@@ -159,17 +161,17 @@ static_assert(CB_COUNT * 8 <= M_BETA && PB_COUNT * 8 <= M_BETA, "barrier area");
 // ---- TMEM columns
 // chain: C1^T (two buffers), C3^T, S'^T (bf16 pairs), D^T (fp16 pairs)
 constexpr uint32_t COL_C1 = 0, COL_C3 = 256, COL_SP = 384, COL_DT = 448;
-constexpr uint32_t COL_P1 = 0, COL_W = 64, COL_AV = 128, COL_Q = 192;                 // prep
+constexpr uint32_t COL_P1 = 0, COL_W = 64;                                           // prep
 constexpr uint32_t TMEM_COLS = 512;
 
 // ---- instruction descriptors (M = 128)
 constexpr uint32_t ID_P1 = idesc_f16(128, 64, 1, 1, 1);      // bf16, A MN-major, B MN-major
 constexpr uint32_t ID_W = idesc_f16(128, 64, 1, 0, 0);       // bf16, K-major / K-major
-constexpr uint32_t ID_AV = idesc_f16(128, 64, 0, 0, 1);      // fp16, K-major / MN-major
-constexpr uint32_t ID_Q = idesc_f16(128, 64, 1, 0, 0);       // bf16
-constexpr uint32_t ID_UVT = idesc_f16(128, 128, 0, 1, 0);      // fp16, A (V) MN-major, B K-major
+constexpr uint32_t ID_UVT = idesc_f16(128, 64, 0, 1, 0);       // fp16, A (V) MN-major, B (T') K-major
 constexpr uint32_t ID_STATE_T = idesc_f16(128, 128, 1, 0, 1);  // bf16, A (S'^T) in TMEM, B MN-major
+constexpr uint32_t ID_STATE_H = idesc_f16(128, 64, 1, 0, 1);   // the same, one 64-column half
 constexpr uint32_t ID_C3T = idesc_f16(128, 128, 0, 0, 0);      // fp16, A (D^T) in TMEM, B K-major
+constexpr uint32_t ID_OQK = idesc_f16(128, 64, 0, 0, 0);       // fp16, A (D^T) in TMEM, B (Aqk) K-major
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 
@@ -320,8 +322,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int i = 0; i < 2; ++i) {
                 mbar_init(BAR(CB_FULL + i), 1);
                 mbar_init(BAR(CB_SFREE + i), 10);
+                mbar_init(BAR(CB_OST_FREE + i), 1);
             }
             mbar_init(BAR(CB_C1_FULL), 1);
+            mbar_init(BAR(CB_O_FULL), 1);
             mbar_init(BAR(CB_C3_FULL), 1);
             mbar_init(BAR(CB_O_READY), 4);
             for (int i = 0; i < NRING; ++i) mbar_init(BAR(CB_READY + i), 1);
@@ -367,13 +371,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (is_chain) {
         // ======================================================================= chain CTA
         if (warp == 0) {
-            // ---- output tiles: staged over the slot's V block (two 64-channel boxes, 128B
-            // swizzle); TMA-stored for full chunks, copied row by row otherwise
+            // ---- output tiles: two staging tiles (each two 64-channel boxes, 128B swizzle);
+            // TMA-stored for full chunks, copied row by row otherwise
             for (int n = 0; n < nch; ++n) {
                 const int sl = n & 1;
                 const int64_t t0 = bos + static_cast<int64_t>(n) * C;
                 const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
-                const uint32_t stage = sbase + CH_SLOT + sl * SET_STRIDE + SET_V;
+                const uint32_t stage = sbase + CH_OST + sl * 16384;
                 if (!wait_bar(BAR(CB_O_READY), n & 1, abort_flag)) break;
                 if (L == C) {
                     if (lane == 0) {
@@ -391,7 +395,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(BAR(CB_SFREE + sl));
+                if (lane == 0) mbar_arrive(BAR(CB_OST_FREE + sl));
             }
             if (lane == 0) bulk_wait0();
             __syncwarp();
@@ -404,9 +408,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (lane == 0) {
                     const unsigned char *src = ring + static_cast<uint64_t>(r) * SET_STRIDE;
                     const uint32_t dst = sbase + CH_SLOT + sl * SET_STRIDE;
-                    mbar_arrive_expect_tx(BAR(CB_FULL + sl), SET_BYTES);
-                    for (uint32_t part = 0; part < 5; ++part)
+                    mbar_arrive_expect_tx(BAR(CB_FULL + sl), SET_TX);
+                    for (uint32_t part = 0; part < 4; ++part)
                         bulk_g2s(dst + part * 16384, src + part * 16384, 16384, BAR(CB_FULL + sl));
+                    bulk_g2s(dst + SET_T, src + SET_T, 16384, BAR(CB_FULL + sl));   // T' and Aqk
                     bulk_g2s(dst + SET_DEC, src + SET_DEC, 512, BAR(CB_FULL + sl));
                 }
                 __syncwarp();
@@ -427,14 +432,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 __syncwarp();
             }
+        } else if (warp == 1) {
+            // ---- intra-chunk output product, C1^T[:, 64..127] += D^T Aqk^T, issued once C3^T
+            // (the other reader of D^T, on the critical path) has completed
+            for (int n = 0; n < nch; ++n) {
+                if (!wait_bar(BAR(CB_C3_FULL), n & 1, abort_flag)) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t slot = sbase + CH_SLOT + (n & 1) * SET_STRIDE;
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16_ts(tmem + COL_C1 + (n & 1) * 128 + 64, tmem + COL_DT + ks * 8,
+                                   smem_desc(slot + SET_AQK + ks * 32, 16, 1024, kSwizzle128), ID_OQK, 1);
+                    mma_commit(BAR(CB_O_FULL));
+                }
+                __syncwarp();
+                // that product was the last reader of the slot's Aqk
+                if (!wait_bar(BAR(CB_O_FULL), n & 1, abort_flag)) break;
+                if (lane == 0) mbar_arrive(BAR(CB_SFREE + (n & 1)));
+                __syncwarp();
+            }
         } else if (warp >= 4) {
             // ---- epilogues: 8 warps. The state is kept transposed: a thread owns S^T[v][j] for
             // one value channel v = TMEM lane 32*(warp%4) + lane and 64 key channels
             // j in [64*half, 64*half + 64). Per chunk (all products accumulate in fp32 TMEM):
-            //   C1^T = V^T [T'; Aqk T']^T + S'^T [-W; Qt]^T   columns 0..63: D^T, 64..127: O^T / scale
-            //   C3^T = D^T Kt                                  S^T <- e^Gl (.) S^T + C3^T
+            //   C1^T = [U^T | 0] + S'^T [-W; Qd]^T       columns 0..63: D^T = (U - W S')^T,
+            //                                            columns 64..127: (Qd S')^T
+            //   C3^T = D^T Kt                            S^T <- e^Gl (.) S^T + C3^T
+            //   C1^T[:, 64..127] += D^T Aqk^T            O = scale (Qd S' + Aqk D)
             // The bf16 state copy S'^T and the fp16 pseudo-values D^T are written straight into
-            // TMEM, where they are the A operands of the next products.
+            // TMEM, where they are the A operands of the next products. Warps of half 0 turn
+            // columns 0..63 into D^T; warps of half 1 write the output of chunk n after the chunk's
+            // closing barrier, while the state product of chunk n + 1 runs.
             const int q4 = warp & 3, half = (warp - 4) >> 2;
             const int v = q4 * 32 + lane;              // value channel = TMEM lane
             const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
@@ -473,7 +501,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_fence_after();
                 for (int ks = 0; ks < 4; ++ks)
                     mma_f16(tmem + COL_C1 + s1 * 128, smem_desc(slot + SET_V + ks * 2048, 8192, 1024, kSwizzle128),
-                            smem_desc(slot + SET_AV + ks * 32, 16, 1024, kSwizzle128), ID_UVT, ks > 0);
+                            smem_desc(slot + SET_T + ks * 32, 16, 1024, kSwizzle128), ID_UVT, ks > 0);
                 return true;
             };
             auto issue_state = [&](int n) {
@@ -481,7 +509,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const uint32_t slot = sbase + CH_SLOT + s1 * SET_STRIDE;
                 tc_fence_after();
                 KDA_TRACE_POINT(n, 13);
-                for (int ks = 0; ks < 8; ++ks)
+                // first K step in two halves: columns 0..63 accumulate onto U^T, columns 64..127
+                // (the output half, not touched by the value-side product) start from zero
+                mma_f16_ts(tmem + COL_C1 + s1 * 128, tmem + COL_SP, smem_desc(slot + SET_W, 16384, 1024, kSwizzle128),
+                           ID_STATE_H, 1);
+                mma_f16_ts(tmem + COL_C1 + s1 * 128 + 64, tmem + COL_SP,
+                           smem_desc(slot + SET_Q, 16384, 1024, kSwizzle128), ID_STATE_H, 0);
+                for (int ks = 1; ks < 8; ++ks)
                     mma_f16_ts(tmem + COL_C1 + s1 * 128, tmem + COL_SP + ks * 8,
                                smem_desc(slot + SET_W + ks * 2048, 16384, 1024, kSwizzle128), ID_STATE_T, 1);
                 mma_commit(BAR(CB_C1_FULL));
@@ -509,10 +543,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!wait_bar(BAR(CB_C1_FULL), n & 1, abort_flag)) break;
                 tc_fence_after();
                 if (tid == 128) KDA_TRACE_POINT(n, 9);
-                const uint32_t acc = tmem + lane_base + COL_C1 + sl * 128 + 64 * half;
                 bool ok = true;
                 if (half == 0) {
-                    // pseudo-values D^T[v][t] -> fp16, two tokens per TMEM column (A operand of C3^T)
+                    // pseudo-values D^T[v][t] -> fp16, two tokens per TMEM column (A operand of
+                    // C3^T and of the intra-chunk output product); the previous chunk's output
+                    // product must have read the old D^T
+                    if (n >= 1 && !wait_bar(BAR(CB_O_FULL), (n - 1) & 1, abort_flag)) break;
+                    const uint32_t acc = tmem + lane_base + COL_C1 + sl * 128;
                     uint32_t r0[32], r1[32];
                     tmem_ld32(acc, r0);
                     tmem_ld32(acc + 32, r1);
@@ -531,34 +568,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     named_bar_sync(3, 128);
                     if (tid == 128) {
                         issue_c3(n);
-                        // the next chunk's value-side product follows C3^T on the tensor pipe; this
+                        // the next chunk's value-side product follows on the tensor pipe; this
                         // thread waits for its slot here, so that the product runs during the C3^T
                         // epilogue rather than ahead of the next state product
                         if (n + 1 < nch) ok = issue_uv(n + 1);
                     }
                     __syncwarp();
-                } else {
-                    // output tile O[t][v] = scale * C1^T[v][64 + t] (bf16), staged over the slot's V
-                    // block (two 64-channel boxes, 128B swizzle) for the store warp
-                    const uint32_t stage = sbase + CH_SLOT + sl * SET_STRIDE + SET_V + (v >> 6) * 8192;
-                    const uint32_t vc = static_cast<uint32_t>(v & 63);
-                    const float sc = p.scale;
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t r[32];
-                        tmem_ld32(acc + 32 * hh, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const uint32_t t = static_cast<uint32_t>(32 * hh + i);
-                            const uint32_t a = stage + t * 128u + ((((vc >> 3) ^ (t & 7u))) << 4) + (vc & 7u) * 2u;
-                            st_shared_u16(a, bf16_bits(sc * __uint_as_float(r[i])));
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(BAR(CB_O_READY));
                 }
                 if (tid == 128) KDA_TRACE_POINT(n, 6);
                 if (!ok) break;
@@ -592,13 +607,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (tid == 128) KDA_TRACE_POINT(n, 7);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(BAR(CB_SFREE + sl));
+                if (lane == 0) mbar_arrive(BAR(CB_SFREE + sl));   // decay reads done
                 if (n + 1 < nch) {
                     named_bar_sync(4, 256);
                     if (tid == 128) issue_state(n + 1);
                     __syncwarp();
                 }
                 if (tid == 128) KDA_TRACE_POINT(n, 11);
+                if (half == 1) {
+                    // output tile O[t][v] = scale * C1^T[v][64 + t] (bf16) -> staging tile `sl`
+                    // (two 64-channel boxes, 128B swizzle) for the store warp
+                    if (!wait_bar(BAR(CB_O_FULL), n & 1, abort_flag)) break;
+                    if (n >= 2 && !wait_bar(BAR(CB_OST_FREE + sl), ((n - 2) >> 1) & 1, abort_flag)) break;
+                    tc_fence_after();
+                    const uint32_t acc = tmem + lane_base + COL_C1 + sl * 128 + 64;
+                    const uint32_t stage = sbase + CH_OST + sl * 16384 + (v >> 6) * 8192;
+                    const uint32_t vc = static_cast<uint32_t>(v & 63);
+                    const float sc = p.scale;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t r[32];
+                        tmem_ld32(acc + 32 * hh, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const uint32_t t = static_cast<uint32_t>(32 * hh + i);
+                            const uint32_t a = stage + t * 128u + ((((vc >> 3) ^ (t & 7u))) << 4) + (vc & 7u) * 2u;
+                            st_shared_u16(a, bf16_bits(sc * __uint_as_float(r[i])));
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(BAR(CB_O_READY));
+                }
             }
             // final state: hT[j][v], coalesced across the warp for each key channel j
             if (p.hT && !*abort_flag) {
@@ -669,7 +711,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     KDA_TRACE_POINT(m, 22);
                     bulk_s2g(set + SET_Q, sbase + PR_AKK, 16384);
                     bulk_s2g(set + SET_V, sbase + PR_STG + STG_V, 16384);
-                    bulk_s2g(set + SET_AV, sbase + PR_AVT, 16384);
+                    bulk_s2g(set + SET_T, sbase + PR_AVT, 8192);
+                    bulk_s2g(set + SET_AQK, sbase + PR_AVT + 8192, 8192);
                     bulk_s2g(set + SET_DEC, misc + M_DEC + (kk & 1) * 512, 512);
                     bulk_commit();
                     bulk_wait_read0();
@@ -686,7 +729,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
         } else if (warp >= 4) {
             // ---- chunk preparation: 8 warps, 256 threads. Outgoing tiles are assembled in
-            // dead workspace: Kt^T over Kc^T, -W^T over Kh^T, Qt^T over the AV operand, UV over A/T.
+            // dead workspace: Kt^T over Kc^T, -W^T over Kh^T, Qd^T over A.
             const int t = tid - 128;
             const int q4 = warp & 3, half = (warp - 4) >> 2;
             const int lrow = q4 * 32 + lane;                 // TMEM lane in the epilogues
@@ -884,8 +927,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             const int jj = half * 4 + j;
                             st_shared_v4(sbase + PR_AVT + sw128(64 + rr, jj), pack_f16(v8[0], v8[1]),
                                          pack_f16(v8[2], v8[3]), pack_f16(v8[4], v8[5]), pack_f16(v8[6], v8[7]));
-                            st_shared_v4(sbase + PR_AQB + sw128(rr, jj), pack_bf16(v8[0], v8[1]),
-                                         pack_bf16(v8[2], v8[3]), pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
                         }
                     }
                     // blocks of T read as zeros by the fixed-length products below
@@ -1053,15 +1094,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int ks = 0; ks < 4; ++ks)
                         mma_f16(tmem + COL_W, smem_desc(sbase + PR_KH + ks * 32, 16, 1024, kSwizzle128),
                                 smem_desc(sbase + PR_TB + ks * 32, 16, 1024, kSwizzle128), ID_W, ks > 0);
-                    // [T'; Aqk] T' (fp16); rows 64..127 (Aqk T') are used
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tmem + COL_AV, smem_desc(sbase + PR_AVT + ks * 32, 16, 1024, kSwizzle128),
-                                smem_desc(sbase + PR_AVT + ks * 2048, 16384, 1024, kSwizzle128), ID_AV, ks > 0);
                     mma_commit(BAR(PB_WAV_DONE));
                     KDA_TRACE_POINT(m, 4);
                 }
+                // -------- Qd = Q e^G = Qh diag(e^Ga) (bf16, over the dead A workspace) while W' runs
+                {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int e = t + 256 * i, rr = e >> 3, jj = e & 7;
+                        const uint4 qv = ld_shared_v4(sbase + PR_QH + sw128(rr, jj));
+                        const float sc = ega_s[rr];
+                        st_shared_v4(sbase + PR_AKK + sw128(rr, jj), pack_bf16(sc * lo_bf(qv.x), sc * hi_bf(qv.x)),
+                                     pack_bf16(sc * lo_bf(qv.y), sc * hi_bf(qv.y)),
+                                     pack_bf16(sc * lo_bf(qv.z), sc * hi_bf(qv.z)),
+                                     pack_bf16(sc * lo_bf(qv.w), sc * hi_bf(qv.w)));
+                    }
+                }
 
-                // -------- S4 epilogues: W (anchored copy; final -W unanchored over Kh^T), Aqk T'
+                // -------- S4 epilogue: W = W' diag(e^Ga), published as -W^T over Kh^T
                 if (!wait_bar(BAR(PB_WAV_DONE), kk & 1, abort_flag)) break;
                 tc_fence_after();
                 if (t == 0) KDA_TRACE_POINT(m, 5);
@@ -1072,75 +1122,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const float sc = -ega_s[lrow];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        float v8[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) v8[e] = __uint_as_float(a[8 * j + e]);
                         const int jj = half * 4 + j;
-                        st_shared_v4(sbase + PR_WP + sw128(lrow, jj), pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]),
-                                     pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
-                        st_shared_v4(sbase + PR_KH + sw128(lrow, jj), pack_bf16(sc * v8[0], sc * v8[1]),
-                                     pack_bf16(sc * v8[2], sc * v8[3]), pack_bf16(sc * v8[4], sc * v8[5]),
-                                     pack_bf16(sc * v8[6], sc * v8[7]));
-                    }
-                    if (lrow >= 64) {
-                        // Aqk T' -> rows 64..127 of the value-side A operand
-                        tmem_ld32(tmem + lane_base + COL_AV + half * 32, a);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int jj = half * 4 + j;
-                            st_shared_v4(sbase + PR_AVT + sw128(lrow, jj),
-                                         pack_f16(__uint_as_float(a[8 * j]), __uint_as_float(a[8 * j + 1])),
-                                         pack_f16(__uint_as_float(a[8 * j + 2]), __uint_as_float(a[8 * j + 3])),
-                                         pack_f16(__uint_as_float(a[8 * j + 4]), __uint_as_float(a[8 * j + 5])),
-                                         pack_f16(__uint_as_float(a[8 * j + 6]), __uint_as_float(a[8 * j + 7])));
-                        }
+                        st_shared_v4(sbase + PR_KH + sw128(lrow, jj),
+                                     pack_bf16(sc * __uint_as_float(a[8 * j]), sc * __uint_as_float(a[8 * j + 1])),
+                                     pack_bf16(sc * __uint_as_float(a[8 * j + 2]), sc * __uint_as_float(a[8 * j + 3])),
+                                     pack_bf16(sc * __uint_as_float(a[8 * j + 4]), sc * __uint_as_float(a[8 * j + 5])),
+                                     pack_bf16(sc * __uint_as_float(a[8 * j + 6]), sc * __uint_as_float(a[8 * j + 7])));
                     }
                 }
+                // hand the finished set to the publisher
                 fence_proxy_async_smem();
                 tc_fence_before();
                 named_bar_sync(2, 256);
                 if (t == 0) {
                     mbar_arrive(BAR(PB_OUTB_READY));
-                    tc_fence_after();
-                    // W'^T Aqk^T (bf16)
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tmem + COL_Q, smem_desc(sbase + PR_WP + ks * 32, 16, 1024, kSwizzle128),
-                                smem_desc(sbase + PR_AQB + ks * 32, 16, 1024, kSwizzle128), ID_Q, ks > 0);
-                    mma_commit(BAR(PB_Q_DONE));
+                    mbar_arrive(BAR(PB_OUTC_READY));
                     KDA_TRACE_POINT(m, 6);
                 }
-
-                // -------- Qt = (Qh - Aqk W') e^Ga, over the dead A workspace (the value side of the
-                // chunk is computed by the chain CTA from V and [T'; Aqk T'])
-                if (!wait_bar(BAR(PB_Q_DONE), kk & 1, abort_flag)) break;
-                tc_fence_after();
-                if (t == 0) KDA_TRACE_POINT(m, 7);
-                {
-                    uint32_t a[32];
-                    tmem_ld32(tmem + lane_base + COL_Q + half * 32, a);
-                    tmem_wait_ld();
-                    const float sc = ega_s[lrow];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int jj = half * 4 + j;
-                        const uint4 qv = ld_shared_v4(sbase + PR_QH + sw128(lrow, jj));
-                        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-                        uint32_t o[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            o[e] = pack_bf16(sc * (lo_bf(qw[e]) - __uint_as_float(a[8 * j + 2 * e])),
-                                             sc * (hi_bf(qw[e]) - __uint_as_float(a[8 * j + 2 * e + 1])));
-                        st_shared_v4(sbase + PR_AKK + sw128(lrow, jj), o[0], o[1], o[2], o[3]);
-                    }
-                    if (t == 0) KDA_TRACE_POINT(m, 14);
-                }
-                if (t == 0) KDA_TRACE_POINT(m, 15);
-                // hand the finished set to the publisher
-                fence_proxy_async_smem();
-                tc_fence_before();
-                named_bar_sync(2, 256);
-                if (t == 0) mbar_arrive(BAR(PB_OUTC_READY));
             }
         }
     }
