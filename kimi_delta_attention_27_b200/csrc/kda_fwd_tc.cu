@@ -59,10 +59,12 @@ __device__ unsigned long long g_kda_cluster_trace[1024 * 8];
     do {                                                                                            \
         if (blockIdx.x / 4 < 1024) g_kda_cluster_trace[(blockIdx.x / 4) * 8 + (slot)] = (value);    \
     } while (0)
-__device__ int g_kda_trace_cluster = 0;   // the cluster whose chunks are timed
+#ifndef KDA_TRACE_CLUSTER_ID
+#define KDA_TRACE_CLUSTER_ID 0   // the cluster whose chunks are timed
+#endif
 #define KDA_TRACE_POINT(chunk, point)                                                               \
     do {                                                                                            \
-        if (static_cast<int>(blockIdx.x / 4) == g_kda_trace_cluster && (chunk) < 64)                \
+        if (blockIdx.x / 4 == KDA_TRACE_CLUSTER_ID && (chunk) < 64)                                 \
             g_kda_trace[(rank * 64 + (chunk)) * 32 + (point)] = ptx::globaltimer();                 \
     } while (0)
 #else
@@ -146,8 +148,9 @@ enum {
 };
 // prep barriers
 enum {
-    PB_STAGE_FULL = 0, PB_STAGE_FREE, PB_VSTAGE_FULL, PB_VSTAGE_FREE, PB_EW_DONE, PB_P1_DONE, PB_SOLVE_DONE,
-    PB_WAV_DONE, PB_WEPI_DONE, PB_Q_DONE,
+    PB_STAGE_FULL = 0, PB_STAGE_FREE, PB_VSTAGE_FULL, PB_VSTAGE_FREE, PB_SPARE4,
+    PB_P1_DONE, PB_SPARE6,
+    PB_WAV_DONE, PB_SPARE8, PB_SPARE9,
     PB_OUTA_READY,      // Kt^T final (over Kc^T)
     PB_OUTB_READY,      // -W^T final (over Kh^T)
     PB_OUTC_READY,      // Qd^T (over A), T' and Aqk, V, e^Gl final
@@ -229,6 +232,12 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
                  : "r"(addr)
                  : "memory");
     return v;
+}
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t x) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(x) : "memory");
+}
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t x) {
     asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(x) : "memory");
@@ -745,6 +754,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 return (t < C && m < nch && tok < eos) ? p.beta[tok * H + h] : 0.f;
             };
             float beta_next = load_beta(first);
+            // the blocks of T' above the diagonal are never written per chunk: clear both T' tiles
+            for (int e = t; e < 512; e += 256) {
+                st_shared_v4(sbase + PR_AVT + e * 16, 0u, 0u, 0u, 0u);   // rows 0..63 (T')
+                st_shared_v4(sbase + PR_TB + e * 16, 0u, 0u, 0u, 0u);
+            }
             int kk = 0;
             for (int m = first; m < nch; m += NPREP, ++kk) {
                 const int64_t t0 = bos + static_cast<int64_t>(m) * C;
@@ -977,6 +991,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     named_bar_sync(2, 256);
                     if (t == 0) KDA_TRACE_POINT(m, 10);
+                    // T' = T diag(beta) is written straight into its two operand tiles as each block of
+                    // T becomes final: fp16 (rows 0..63 of the [T'; Aqk] tile) and bf16 (TB); the blocks
+                    // above the diagonal are zero and were cleared once.
+                    // address of T'[r][c..] (c a multiple of 2) in a K-major 128B-swizzled fp16/bf16 tile
+                    auto tp_addr = [&](uint32_t base, int r, int c) -> uint32_t {
+                        return base + sw128(static_cast<uint32_t>(r), static_cast<uint32_t>(c >> 3)) +
+                               static_cast<uint32_t>(c & 7) * 2u;
+                    };
                     // (b) blocks (1,0) and (3,2): P = A_IJ T_JJ, then T_IJ = -T_II P (two columns per thread)
                     {
                         const int blk = t >> 7, rr = (t >> 3) & 15, cc = (t & 7) * 2;
@@ -996,6 +1018,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             }
                         }
                         *reinterpret_cast<float2 *>(P + blk * 256 + rr * 16 + cc) = make_float2(p0, p1);
+                        // T' of the diagonal blocks (final since (a)): row t >> 2, 4 columns
+                        {
+                            const int r = t >> 2, cq = (t & 3) * 4, c = (r & ~15) + cq;
+                            const float4 tv = *reinterpret_cast<const float4 *>(T + r * AKK_LD + c);
+                            const float4 bv = *reinterpret_cast<const float4 *>(beta_s + c);
+                            const float x0 = tv.x * bv.x, x1 = tv.y * bv.y, x2 = tv.z * bv.z, x3 = tv.w * bv.w;
+                            st_shared_v2(tp_addr(sbase + PR_AVT, r, c), pack_f16(x0, x1), pack_f16(x2, x3));
+                            st_shared_v2(tp_addr(sbase + PR_TB, r, c), pack_bf16(x0, x1), pack_bf16(x2, x3));
+                        }
                         named_bar_sync(2, 256);
                         const float *trow = T + (16 * I + rr) * AKK_LD + 16 * I;
                         p0 = 0.f;
@@ -1012,6 +1043,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             }
                         }
                         *reinterpret_cast<float2 *>(T + (16 * I + rr) * AKK_LD + 16 * J + cc) = make_float2(-p0, -p1);
+                        const int r = 16 * I + rr, c = 16 * J + cc;
+                        const float x0 = -p0 * beta_s[c], x1 = -p1 * beta_s[c + 1];
+                        st_shared_u32(tp_addr(sbase + PR_AVT, r, c), pack_f16(x0, x1));
+                        st_shared_u32(tp_addr(sbase + PR_TB, r, c), pack_bf16(x0, x1));
                     }
                     named_bar_sync(2, 256);
                     if (t == 0) KDA_TRACE_POINT(m, 11);
@@ -1058,31 +1093,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                 p3 = fmaf(t4[e], pv.w, p3);
                             }
                         }
-                        *reinterpret_cast<float4 *>(T + (32 + rr) * AKK_LD + c4) = make_float4(-p0, -p1, -p2, -p3);
+                        // final block of T; T itself is not read again, only T' is written
+                        const float4 bv = *reinterpret_cast<const float4 *>(beta_s + c4);
+                        const float x0 = -p0 * bv.x, x1 = -p1 * bv.y, x2 = -p2 * bv.z, x3 = -p3 * bv.w;
+                        st_shared_v2(tp_addr(sbase + PR_AVT, 32 + rr, c4), pack_f16(x0, x1), pack_f16(x2, x3));
+                        st_shared_v2(tp_addr(sbase + PR_TB, 32 + rr, c4), pack_bf16(x0, x1), pack_bf16(x2, x3));
                     }
-                    named_bar_sync(2, 256);
                     if (t == 0) KDA_TRACE_POINT(m, 12);
-                    // T' = T diag(beta): fp16 -> AV rows 0..63, bf16 -> TB
-                    {
-                        const int rr = t >> 2, qt = t & 3;
-#pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {
-                            const int j = qt * 2 + jj;
-                            const float4 ta = *reinterpret_cast<const float4 *>(T + rr * AKK_LD + 8 * j);
-                            const float4 tb = *reinterpret_cast<const float4 *>(T + rr * AKK_LD + 8 * j + 4);
-                            const float4 ba = *reinterpret_cast<const float4 *>(beta_s + 8 * j);
-                            const float4 bb = *reinterpret_cast<const float4 *>(beta_s + 8 * j + 4);
-                            const float tvv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-                            const float bvv[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
-                            float v8[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) v8[e] = (8 * j + e) <= rr ? tvv[e] * bvv[e] : 0.f;
-                            st_shared_v4(sbase + PR_AVT + sw128(rr, j), pack_f16(v8[0], v8[1]), pack_f16(v8[2], v8[3]),
-                                         pack_f16(v8[4], v8[5]), pack_f16(v8[6], v8[7]));
-                            st_shared_v4(sbase + PR_TB + sw128(rr, j), pack_bf16(v8[0], v8[1]),
-                                         pack_bf16(v8[2], v8[3]), pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
-                        }
-                    }
                 }
                 if (t == 0) KDA_TRACE_POINT(m, 16);
                 fence_proxy_async_smem();
@@ -1306,9 +1323,6 @@ cudaError_t launch_fwd_tc_noalloc(const FwdParams &p, int64_t rows, cudaStream_t
 #ifdef KDA_TRACE
 extern "C" int kda_trace_read(unsigned long long *host) {
     return static_cast<int>(cudaMemcpyFromSymbol(host, g_kda_trace, sizeof(g_kda_trace)));
-}
-extern "C" int kda_trace_set_cluster(int c) {
-    return static_cast<int>(cudaMemcpyToSymbol(g_kda_trace_cluster, &c, sizeof(int)));
 }
 extern "C" int kda_trace_read_clusters(unsigned long long *host) {
     return static_cast<int>(cudaMemcpyFromSymbol(host, g_kda_cluster_trace, sizeof(g_kda_cluster_trace)));
