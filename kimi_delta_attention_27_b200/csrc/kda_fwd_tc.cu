@@ -128,6 +128,10 @@ static_assert(PR_AVT % 1024 == 0 && PR_AKK % 1024 == 0 && PR_KH % 1024 == 0 &&
 // misc area (offsets from the misc base of either role)
 constexpr uint32_t M_BAR = 0;                      // up to 32 barriers
 constexpr uint32_t M_BETA = 256, M_EGA = 512;                  // 64, 128 floats
+// prep: beta of the two staged chunks (2 x 64 floats), the chunk index of the last four local
+// chunks, the number of chunks the chain CTA has pulled (written by the chain CTA);
+// chain: the next chunk to hand out (incremented by the prep CTAs)
+constexpr uint32_t M_BETAQ = 1024, M_CHUNKQ = 1536, M_CONSUMED = 1552, M_NEXT = 1568;
 constexpr uint32_t M_DEC = 2048;                               // 2 x 128 floats (e^Gl, part of the set)
 constexpr uint32_t M_TMEM = 3072, M_ABORT = 3088, M_SMID = 3104;
 constexpr uint32_t MISC_BYTES = 3584;
@@ -152,9 +156,9 @@ enum {
     PB_P1_DONE, PB_SPARE6,
     PB_WAV_DONE, PB_SPARE8, PB_SPARE9,
     PB_OUTA_READY,      // Kt^T final (over Kc^T)
-    PB_OUTB_READY,      // -W^T final (over Kh^T)
+    PB_OUTB_READY,      // -W^T final (over the fp32 T workspace)
     PB_OUTC_READY,      // Qd^T (over A), T' and Aqk, V, e^Gl final
-    PB_OUTAB_FREE,      // publisher has read parts A and B out
+    PB_OUTA_FREE,       // publisher has read part A out
     PB_OUTC_FREE,       // publisher has read part C out
     PB_RING_FREE = 15,  // NRING: ring slot released by the chain CTA (remote arrival)
     PB_COUNT = PB_RING_FREE + NRING
@@ -279,6 +283,48 @@ __device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr) {
     asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
     return v;
 }
+// named barrier that also ORs a predicate over the participating threads: every thread gets the
+// same answer, so a loop left on it is left by all of them (no thread is stranded at a barrier)
+__device__ __forceinline__ bool named_bar_any(uint32_t id, uint32_t nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, %3, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+// atomic add on a u32 in shared memory of a cluster CTA (shared::cluster address); returns the old value
+__device__ __forceinline__ uint32_t atom_add_cluster(uint32_t addr, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ void st_release_cluster(uint32_t addr, uint32_t v) {
+    asm volatile("st.release.cluster.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_cta(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+// bounded wait until the u32 at `addr` (this CTA's shared memory) reaches `target`
+__device__ __forceinline__ bool wait_count(uint32_t addr, uint32_t target, volatile uint32_t *abort_flag) {
+    if (ld_acquire_cta(addr) >= target) return true;
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+        if (ld_acquire_cta(addr) >= target) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(&g_kda_device_error, 1u);
+            return false;
+        }
+    }
+}
+
 __device__ __forceinline__ uint32_t smid() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
@@ -340,10 +386,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int i = 0; i < NRING; ++i) mbar_init(BAR(CB_READY + i), 1);
             const uint32_t sm = smid();
             *reinterpret_cast<volatile uint32_t *>(miscg + M_SMID) = sm;
+            *reinterpret_cast<volatile uint32_t *>(miscg + M_NEXT) = 0u;
             *abort_flag = sm < static_cast<uint32_t>(kMaxRings) ? 0u : 1u;
             if (sm >= static_cast<uint32_t>(kMaxRings)) atomicOr(&g_kda_device_error, 2u);
         } else {
-            for (int i = 0; i < PB_RING_FREE; ++i) mbar_init(BAR(i), 1);
+            for (int i = 0; i < PB_RING_FREE; ++i) mbar_init(BAR(i), i == PB_STAGE_FULL ? 2 : 1);
+            *reinterpret_cast<volatile uint32_t *>(miscg + M_CONSUMED) = 0u;
             for (int i = 0; i < NRING; ++i) mbar_init(BAR(PB_RING_FREE + i), 1);
             *abort_flag = 0;
         }
@@ -434,8 +482,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!wait_bar(BAR(CB_FULL + sl), (n >> 1) & 1, abort_flag)) break;
                 if (lane == 0) {
                     if (n + NRING < nch) {
-                        const uint32_t prod = 1u + static_cast<uint32_t>(n % NPREP);
-                        mbar_arrive_remote(mapa(sbase + PR_MISC + M_BAR + 8u * (PB_RING_FREE + n % NRING), prod));
+                        // chunks 0..n have been pulled: any prep CTA may reuse the slot of chunk n
+                        for (uint32_t pr = 1; pr <= static_cast<uint32_t>(NPREP); ++pr)
+                            st_release_cluster(mapa(sbase + PR_MISC + M_CONSUMED, pr), static_cast<uint32_t>(n + 1));
                     }
                     mbar_arrive(BAR(CB_SFREE + sl));
                 }
@@ -549,7 +598,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             __syncwarp();
             for (int n = 0; n < nch; ++n) {
                 const int sl = n & 1;
-                if (!wait_bar(BAR(CB_C1_FULL), n & 1, abort_flag)) break;
+                // A wait that gives up (abort) does not leave the loop on its own: the warps leave
+                // together at the chunk's closing barrier.
+                wait_bar(BAR(CB_C1_FULL), n & 1, abort_flag);
                 tc_fence_after();
                 if (tid == 128) KDA_TRACE_POINT(n, 9);
                 bool ok = true;
@@ -557,7 +608,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     // pseudo-values D^T[v][t] -> fp16, two tokens per TMEM column (A operand of
                     // C3^T and of the intra-chunk output product); the previous chunk's output
                     // product must have read the old D^T
-                    if (n >= 1 && !wait_bar(BAR(CB_O_FULL), (n - 1) & 1, abort_flag)) break;
+                    if (n >= 1) wait_bar(BAR(CB_O_FULL), (n - 1) & 1, abort_flag);
                     const uint32_t acc = tmem + lane_base + COL_C1 + sl * 128;
                     uint32_t r0[32], r1[32];
                     tmem_ld32(acc, r0);
@@ -585,8 +636,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     __syncwarp();
                 }
                 if (tid == 128) KDA_TRACE_POINT(n, 6);
-                if (!ok) break;
-                if (!wait_bar(BAR(CB_C3_FULL), n & 1, abort_flag)) break;
+                (void)ok;
+                wait_bar(BAR(CB_C3_FULL), n & 1, abort_flag);
                 tc_fence_after();
                 if (tid == 128) KDA_TRACE_POINT(n, 10);
                 {
@@ -618,7 +669,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(BAR(CB_SFREE + sl));   // decay reads done
                 if (n + 1 < nch) {
-                    named_bar_sync(4, 256);
+                    if (named_bar_any(4, 256, *abort_flag != 0)) break;
                     if (tid == 128) issue_state(n + 1);
                     __syncwarp();
                 }
@@ -626,8 +677,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (half == 1) {
                     // output tile O[t][v] = scale * C1^T[v][64 + t] (bf16) -> staging tile `sl`
                     // (two 64-channel boxes, 128B swizzle) for the store warp
-                    if (!wait_bar(BAR(CB_O_FULL), n & 1, abort_flag)) break;
-                    if (n >= 2 && !wait_bar(BAR(CB_OST_FREE + sl), ((n - 2) >> 1) & 1, abort_flag)) break;
+                    wait_bar(BAR(CB_O_FULL), n & 1, abort_flag);
+                    if (n >= 2) wait_bar(BAR(CB_OST_FREE + sl), ((n - 2) >> 1) & 1, abort_flag);
                     tc_fence_after();
                     const uint32_t acc = tmem + lane_base + COL_C1 + sl * 128 + 64;
                     const uint32_t stage = sbase + CH_OST + sl * 16384 + (v >> 6) * 8192;
@@ -666,20 +717,43 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     } else {
         // ======================================================================= prep CTA
-        const int first = static_cast<int>(rank) - 1;   // chunks first, first + 3, ...
         if (warp == 0) {
-            // ---- q, k, g staging loads
-            int kk = 0;
-            for (int m = first; m < nch; m += NPREP, ++kk) {
-                const int32_t row = static_cast<int32_t>(bos + static_cast<int64_t>(m) * C);
+            // ---- chunk hand-out and staging loads. The prep CTAs take chunks from a counter in
+            // the chain CTA's shared memory, so a slower CTA simply prepares fewer of them. For
+            // each local chunk kk: the chunk index (queue of 4), its beta (queue of 2), q, k, g by
+            // TMA, then v.
+            volatile uint32_t *chunkq = reinterpret_cast<volatile uint32_t *>(miscg + M_CHUNKQ);
+            for (int kk = 0;; ++kk) {
                 if (kk >= 1 && !wait_bar(BAR(PB_STAGE_FREE), (kk - 1) & 1, abort_flag)) break;
+                uint32_t mm = 0;
+                if (lane == 0) mm = atom_add_cluster(mapa(sbase + CH_MISC + M_NEXT, 0), 1u);
+                mm = __shfl_sync(0xffffffffu, mm, 0);
+                const int m = static_cast<int>(mm);
+                if (lane == 0) chunkq[kk & 3] = mm;
+                if (m >= nch) {
+                    // no chunk left: release the other roles of this CTA
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(BAR(PB_STAGE_FULL));
+                        mbar_arrive(BAR(PB_STAGE_FULL));
+                    }
+                    break;
+                }
+                const int64_t t0 = bos + static_cast<int64_t>(m) * C;
+                const int32_t row = static_cast<int32_t>(t0);
                 if (lane == 0) {
                     mbar_arrive_expect_tx(BAR(PB_STAGE_FULL), STAGE_TX);
                     tma_load_3d(sbase + PR_STG + STG_Q, &maps.q, BAR(PB_STAGE_FULL), 0, h, row);
                     tma_load_3d(sbase + PR_STG + STG_K, &maps.k, BAR(PB_STAGE_FULL), 0, h, row);
                     tma_load_3d(sbase + PR_STG + STG_G, &maps.g, BAR(PB_STAGE_FULL), 0, h, row);
                 }
+                float *betaq = reinterpret_cast<float *>(miscg + M_BETAQ) + (kk & 1) * C;
+                for (int i = lane; i < C; i += 32) {
+                    const int64_t tok = t0 + i;
+                    betaq[i] = tok < eos ? p.beta[tok * H + h] : 0.f;
+                }
                 __syncwarp();
+                if (lane == 0) mbar_arrive(BAR(PB_STAGE_FULL));   // second arrival: index and beta stored
                 if (kk >= 1 && !wait_bar(BAR(PB_VSTAGE_FREE), (kk - 1) & 1, abort_flag)) break;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(BAR(PB_VSTAGE_FULL), VSTAGE_TX);
@@ -691,28 +765,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         } else if (warp == 3) {
             // ---- publisher: finished parts of the operand set (smem) -> ring slot (global),
             // each by bulk stores as soon as the part is final
-            int kk = 0;
-            for (int m = first; m < nch; m += NPREP, ++kk) {
+            volatile uint32_t *chunkq = reinterpret_cast<volatile uint32_t *>(miscg + M_CHUNKQ);
+            for (int kk = 0;; ++kk) {
+                // part A of the local chunk kk is final (or, past the last chunk, the end signal)
+                if (!wait_bar(BAR(PB_OUTA_READY), kk & 1, abort_flag)) break;
+                const int m = static_cast<int>(chunkq[kk & 3]);
+                if (m >= nch) break;
                 const int r = m % NRING;
                 unsigned char *set = ring + static_cast<uint64_t>(r) * SET_STRIDE;
                 // the ring slot must have been pulled by the chain CTA (chunk m - NRING)
-                if (m >= NRING && !wait_bar(BAR(PB_RING_FREE + r), ((m / NRING) - 1) & 1, abort_flag)) break;
+                if (m >= NRING && !wait_count(misc + M_CONSUMED, static_cast<uint32_t>(m - NRING + 1), abort_flag))
+                    break;
                 if (lane == 0) KDA_TRACE_POINT(m, 18);
-                if (!wait_bar(BAR(PB_OUTA_READY), kk & 1, abort_flag)) break;
                 if (lane == 0) {
                     KDA_TRACE_POINT(m, 19);
                     bulk_s2g(set + SET_KT, sbase + PR_KC, 16384);
                     bulk_commit();
+                    bulk_wait_read0();
+                    mbar_arrive(BAR(PB_OUTA_FREE));   // Kc^T / Kt^T may be overwritten
                 }
                 __syncwarp();
                 if (!wait_bar(BAR(PB_OUTB_READY), kk & 1, abort_flag)) break;
                 if (lane == 0) {
                     KDA_TRACE_POINT(m, 20);
-                    bulk_s2g(set + SET_W, sbase + PR_KH, 16384);
+                    bulk_s2g(set + SET_W, sbase + PR_T, 16384);
                     bulk_commit();
-                    bulk_wait_read0();
                     KDA_TRACE_POINT(m, 21);
-                    mbar_arrive(BAR(PB_OUTAB_FREE));
                 }
                 __syncwarp();
                 if (!wait_bar(BAR(PB_OUTC_READY), kk & 1, abort_flag)) break;
@@ -744,32 +822,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int lrow = q4 * 32 + lane;                 // TMEM lane in the epilogues
             const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
             float *wsf = reinterpret_cast<float *>(sgen);
-            float *beta_s = reinterpret_cast<float *>(miscg + M_BETA);
             float *ega_s = reinterpret_cast<float *>(miscg + M_EGA);
             float *dec_all = reinterpret_cast<float *>(miscg + M_DEC);
-            // beta of chunk m (0 past the sequence end), loaded one chunk of this CTA ahead so
-            // that its global-memory latency is hidden behind the previous chunk's work
-            auto load_beta = [&](int m) -> float {
-                const int64_t tok = bos + static_cast<int64_t>(m) * C + t;
-                return (t < C && m < nch && tok < eos) ? p.beta[tok * H + h] : 0.f;
-            };
-            float beta_next = load_beta(first);
+            volatile uint32_t *chunkq = reinterpret_cast<volatile uint32_t *>(miscg + M_CHUNKQ);
             // the blocks of T' above the diagonal are never written per chunk: clear both T' tiles
             for (int e = t; e < 512; e += 256) {
                 st_shared_v4(sbase + PR_AVT + e * 16, 0u, 0u, 0u, 0u);   // rows 0..63 (T')
                 st_shared_v4(sbase + PR_TB + e * 16, 0u, 0u, 0u, 0u);
             }
-            int kk = 0;
-            for (int m = first; m < nch; m += NPREP, ++kk) {
+            // A wait that gives up (abort) does not leave the loop on its own: the 8 warps leave
+            // together at the next named barrier, which ORs the abort flag over them.
+            for (int kk = 0;; ++kk) {
+#ifdef KDA_TRACE
+                const unsigned long long trace_start = globaltimer();
+#endif
+                // part A of the previous set (over Kc^T) must have been read out by the publisher;
+                // part B (over T) is covered by the wait for part C before T is next written
+                if (kk >= 1) wait_bar(BAR(PB_OUTA_FREE), (kk - 1) & 1, abort_flag);
+                wait_bar(BAR(PB_STAGE_FULL), kk & 1, abort_flag);
+                const int m = static_cast<int>(chunkq[kk & 3]);   // this CTA's kk-th chunk
+                const bool no_chunk = m >= nch;
+                if (named_bar_any(2, 256, no_chunk || *abort_flag != 0)) {
+                    if (t == 0) mbar_arrive(BAR(PB_OUTA_READY));   // the publisher's end signal
+                    break;
+                }
                 const int64_t t0 = bos + static_cast<int64_t>(m) * C;
                 const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
-                if (*abort_flag) break;
-                if (t == 0) KDA_TRACE_POINT(m, 0);
-                if (t < C) beta_s[t] = beta_next;
-                beta_next = load_beta(m + NPREP);
-                // parts A and B of the previous set must have been read out by the publisher
-                if (kk >= 1 && !wait_bar(BAR(PB_OUTAB_FREE), (kk - 1) & 1, abort_flag)) break;
-                if (!wait_bar(BAR(PB_STAGE_FULL), kk & 1, abort_flag)) break;
+                const float *beta_s = reinterpret_cast<const float *>(miscg + M_BETAQ) + (kk & 1) * C;
+#ifdef KDA_TRACE
+                if (t == 0 && blockIdx.x / 4 == KDA_TRACE_CLUSTER_ID && m < 64)
+                    g_kda_trace[(rank * 64 + m) * 32 + 0] = trace_start;
+#endif
                 if (t == 0) KDA_TRACE_POINT(m, 1);
 
                 // -------- S1: running log-decay and the anchored factors. A thread owns a pair of
@@ -796,7 +879,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     // row-quarter sums of g per channel, [4][128] floats in the solve's scratch
                     float *gq = reinterpret_cast<float *>(sgen + PR_P);
                     *reinterpret_cast<float2 *>(gq + tq * 128 + c0) = make_float2(px, py);
-                    named_bar_sync(2, 256);
+                    if (named_bar_any(2, 256, *abort_flag != 0)) break;
                     float2 qs[4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) qs[q] = *reinterpret_cast<const float2 *>(gq + q * 128 + c0);
@@ -868,7 +951,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                 }
                 fence_proxy_async_smem();
-                named_bar_sync(2, 256);
+                if (named_bar_any(2, 256, *abort_flag != 0)) break;
                 // The prep MMAs are issued by this thread right after the barrier that ends the
                 // phase writing their operands (no hop through another warp).
                 if (t == 0) {
@@ -882,7 +965,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     KDA_TRACE_POINT(m, 2);
                 }
                 // value tile bf16 -> fp16 in place (B operand of the value-side MMA)
-                if (!wait_bar(BAR(PB_VSTAGE_FULL), kk & 1, abort_flag)) break;
+                wait_bar(BAR(PB_VSTAGE_FULL), kk & 1, abort_flag);
 #pragma unroll
                 for (int c2 = 0; c2 < 4; ++c2) {
                     const uint32_t a = sbase + PR_STG + STG_V + (t + 256 * c2) * 16;
@@ -894,8 +977,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
                 // -------- S2 epilogue: A (fp32, masked, beta-scaled) and Aqk (fp16 + bf16); Kt^T out
                 // (part C of the previous set, over A / T and the AV operand, must be read out)
-                if (kk >= 1 && !wait_bar(BAR(PB_OUTC_FREE), (kk - 1) & 1, abort_flag)) break;
-                if (!wait_bar(BAR(PB_P1_DONE), kk & 1, abort_flag)) break;
+                if (kk >= 1) wait_bar(BAR(PB_OUTC_FREE), (kk - 1) & 1, abort_flag);
+                wait_bar(BAR(PB_P1_DONE), kk & 1, abort_flag);
                 tc_fence_after();
                 if (t == 0) KDA_TRACE_POINT(m, 3);
                 {
@@ -950,7 +1033,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                named_bar_sync(2, 256);
+                if (named_bar_any(2, 256, *abort_flag != 0)) break;
                 if (t == 0) {
                     mbar_arrive(BAR(PB_OUTA_READY));
                     KDA_TRACE_POINT(m, 9);
@@ -989,7 +1072,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             for (int rr = 0; rr < 16; ++rr) T[(16 * wb + rr) * AKK_LD + 16 * wb + li] = x[rr];
                         }
                     }
-                    named_bar_sync(2, 256);
+                    if (named_bar_any(2, 256, *abort_flag != 0)) break;
                     if (t == 0) KDA_TRACE_POINT(m, 10);
                     // T' = T diag(beta) is written straight into its two operand tiles as each block of
                     // T becomes final: fp16 (rows 0..63 of the [T'; Aqk] tile) and bf16 (TB); the blocks
@@ -1027,7 +1110,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             st_shared_v2(tp_addr(sbase + PR_AVT, r, c), pack_f16(x0, x1), pack_f16(x2, x3));
                             st_shared_v2(tp_addr(sbase + PR_TB, r, c), pack_bf16(x0, x1), pack_bf16(x2, x3));
                         }
-                        named_bar_sync(2, 256);
+                        if (named_bar_any(2, 256, *abort_flag != 0)) break;
                         const float *trow = T + (16 * I + rr) * AKK_LD + 16 * I;
                         p0 = 0.f;
                         p1 = 0.f;
@@ -1048,7 +1131,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         st_shared_u32(tp_addr(sbase + PR_AVT, r, c), pack_f16(x0, x1));
                         st_shared_u32(tp_addr(sbase + PR_TB, r, c), pack_bf16(x0, x1));
                     }
-                    named_bar_sync(2, 256);
+                    if (named_bar_any(2, 256, *abort_flag != 0)) break;
                     if (t == 0) KDA_TRACE_POINT(m, 11);
                     // (c) rows 32..63, columns 0..31: P2 = A[32:, :32] T[:32, :32]; T = -T[32:, 32:] P2.
                     // Lane = row, warp = 4-column group, so the T and P2 reads are warp-uniform
@@ -1075,7 +1158,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         }
                         *reinterpret_cast<float4 *>(P + rr * 32 + (((c4 >> 2) ^ (rr & 7)) << 2)) =
                             make_float4(p0, p1, p2, p3);
-                        named_bar_sync(2, 256);
+                        if (named_bar_any(2, 256, *abort_flag != 0)) break;
                         const float *trow = T + (32 + rr) * AKK_LD + 32;
                         p0 = p1 = p2 = p3 = 0.f;
 #pragma unroll
@@ -1104,7 +1187,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (t == 0) KDA_TRACE_POINT(m, 16);
                 fence_proxy_async_smem();
                 if (t == 0) KDA_TRACE_POINT(m, 17);
-                named_bar_sync(2, 256);
+                if (named_bar_any(2, 256, *abort_flag != 0)) break;
                 if (t == 0) {
                     tc_fence_after();
                     // W'^T = Kh^T T'^T (bf16)
@@ -1128,8 +1211,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                 }
 
-                // -------- S4 epilogue: W = W' diag(e^Ga), published as -W^T over Kh^T
-                if (!wait_bar(BAR(PB_WAV_DONE), kk & 1, abort_flag)) break;
+                // -------- S4 epilogue: W = W' diag(e^Ga), published as -W^T over the dead fp32 T
+                // (so that the next chunk may overwrite Kh at once)
+                wait_bar(BAR(PB_WAV_DONE), kk & 1, abort_flag);
                 tc_fence_after();
                 if (t == 0) KDA_TRACE_POINT(m, 5);
                 {
@@ -1140,7 +1224,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int jj = half * 4 + j;
-                        st_shared_v4(sbase + PR_KH + sw128(lrow, jj),
+                        st_shared_v4(sbase + PR_T + sw128(lrow, jj),
                                      pack_bf16(sc * __uint_as_float(a[8 * j]), sc * __uint_as_float(a[8 * j + 1])),
                                      pack_bf16(sc * __uint_as_float(a[8 * j + 2]), sc * __uint_as_float(a[8 * j + 3])),
                                      pack_bf16(sc * __uint_as_float(a[8 * j + 4]), sc * __uint_as_float(a[8 * j + 5])),
@@ -1150,7 +1234,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // hand the finished set to the publisher
                 fence_proxy_async_smem();
                 tc_fence_before();
-                named_bar_sync(2, 256);
+                if (named_bar_any(2, 256, *abort_flag != 0)) break;
                 if (t == 0) {
                     mbar_arrive(BAR(PB_OUTB_READY));
                     mbar_arrive(BAR(PB_OUTC_READY));
