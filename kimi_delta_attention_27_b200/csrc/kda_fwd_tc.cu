@@ -20,12 +20,12 @@
 //  * rank 0 ("chain") owns the whole fp32 state (128 x 128) and runs the sequential
 //    part, S5-S7 (and U = T' V), with 128-column MMAs: the dependent-step latency of a
 //    tcgen05 MMA barely depends on N up to 128, so the state is not split.
-//  * ranks 1-3 ("prep") each prepare every third chunk (S0-S4: gates, decayed
-//    blocks, UT solve, W, Qd, Kt), writing the finished 80.5 KB operand set
-//    into a per-cluster ring of 6 slots in global memory (it stays in L2); the
-//    chain CTA pulls each set with one TMA bulk load. Shared memory of another
-//    CTA (DSMEM) carries only barrier signals: its bulk bandwidth is a fraction
-//    of an L2 TMA load's.
+//  * ranks 1-3 ("prep") take chunks from a counter in the chain CTA's shared
+//    memory and prepare them (S0-S4: gates, decayed blocks, UT solve, W, Qd, Kt),
+//    writing each finished 80.5 KB operand set into a per-cluster ring of 6 slots
+//    in global memory (it stays in L2); the chain CTA pulls each set with TMA bulk
+//    loads. Shared memory of another CTA (DSMEM) carries only barrier signals and
+//    counters: its bulk bandwidth is a fraction of an L2 TMA load's.
 //  Every input byte is read from HBM once (q, k, v, g, beta by a prep CTA) and
 //  every output byte written once (by the chain CTA).
 //
@@ -224,6 +224,24 @@ __device__ __forceinline__ float ex2_approx(float y) {
 
 // byte offset of 16-byte chunk j of row r in a tile of 128-byte rows, 128B swizzle
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t j) { return r * 128u + ((j ^ (r & 7u)) << 4); }
+
+// packed fp32 pairs (sm_100 f32x2 instructions): one instruction for both lanes of a float2
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
@@ -780,9 +798,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (lane == 0) {
                     KDA_TRACE_POINT(m, 19);
                     bulk_s2g(set + SET_KT, sbase + PR_KC, 16384);
+                    bulk_s2g(set + SET_V, sbase + PR_STG + STG_V, 16384);
                     bulk_commit();
                     bulk_wait_read0();
-                    mbar_arrive(BAR(PB_OUTA_FREE));   // Kc^T / Kt^T may be overwritten
+                    mbar_arrive(BAR(PB_OUTA_FREE));     // Kt^T may be overwritten
+                    mbar_arrive(BAR(PB_VSTAGE_FREE));   // the next value tile may be loaded
                 }
                 __syncwarp();
                 if (!wait_bar(BAR(PB_OUTB_READY), kk & 1, abort_flag)) break;
@@ -797,7 +817,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (lane == 0) {
                     KDA_TRACE_POINT(m, 22);
                     bulk_s2g(set + SET_Q, sbase + PR_AKK, 16384);
-                    bulk_s2g(set + SET_V, sbase + PR_STG + STG_V, 16384);
                     bulk_s2g(set + SET_T, sbase + PR_AVT, 8192);
                     bulk_s2g(set + SET_AQK, sbase + PR_AVT + 8192, 8192);
                     bulk_s2g(set + SET_DEC, misc + M_DEC + (kk & 1) * 512, 512);
@@ -805,7 +824,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     bulk_wait_read0();
                     KDA_TRACE_POINT(m, 23);
                     mbar_arrive(BAR(PB_OUTC_FREE));
-                    mbar_arrive(BAR(PB_VSTAGE_FREE));
                     bulk_wait0();
                     KDA_TRACE_POINT(m, 24);
                     fence_proxy_async_global();
@@ -816,7 +834,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
         } else if (warp >= 4) {
             // ---- chunk preparation: 8 warps, 256 threads. Outgoing tiles are assembled in
-            // dead workspace: Kt^T over Kc^T, -W^T over Kh^T, Qd^T over A.
+            // dead workspace: Kt^T over Kc^T, -W^T over the fp32 T, Qd^T over the fp32 A.
             const int t = tid - 128;
             const int q4 = warp & 3, half = (warp - 4) >> 2;
             const int lrow = q4 * 32 + lane;                 // TMEM lane in the epilogues
@@ -839,7 +857,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // part A of the previous set (over Kc^T) must have been read out by the publisher;
                 // part B (over T) is covered by the wait for part C before T is next written
                 if (kk >= 1) wait_bar(BAR(PB_OUTA_FREE), (kk - 1) & 1, abort_flag);
+#ifdef KDA_TRACE
+                const unsigned long long trace_afree = globaltimer();
+#endif
                 wait_bar(BAR(PB_STAGE_FULL), kk & 1, abort_flag);
+#ifdef KDA_TRACE
+                const unsigned long long trace_sfull = globaltimer();
+#endif
                 const int m = static_cast<int>(chunkq[kk & 3]);   // this CTA's kk-th chunk
                 const bool no_chunk = m >= nch;
                 if (named_bar_any(2, 256, no_chunk || *abort_flag != 0)) {
@@ -850,8 +874,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
                 const float *beta_s = reinterpret_cast<const float *>(miscg + M_BETAQ) + (kk & 1) * C;
 #ifdef KDA_TRACE
-                if (t == 0 && blockIdx.x / 4 == KDA_TRACE_CLUSTER_ID && m < 64)
+                if (t == 0 && blockIdx.x / 4 == KDA_TRACE_CLUSTER_ID && m < 64) {
                     g_kda_trace[(rank * 64 + m) * 32 + 0] = trace_start;
+                    g_kda_trace[(rank * 64 + m) * 32 + 25] = trace_afree;
+                    g_kda_trace[(rank * 64 + m) * 32 + 26] = trace_sfull;
+                }
 #endif
                 if (t == 0) KDA_TRACE_POINT(m, 1);
 
@@ -867,32 +894,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const float *gst = reinterpret_cast<const float *>(sgen + PR_STG + STG_G);
                     const uint32_t *qst = reinterpret_cast<const uint32_t *>(sgen + PR_STG + STG_Q);
                     const uint32_t *kst = reinterpret_cast<const uint32_t *>(sgen + PR_STG + STG_K);
+                    // g of the channel pair in log2 units (x, y = channels c0, c0 + 1)
+                    const float2 l2e = make_float2(kLog2e, kLog2e);
                     float2 gv[16];
-                    float px = 0.f, py = 0.f;
+                    float2 ps = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int rr = r0 + i;
-                        gv[i] = rr < L ? *reinterpret_cast<const float2 *>(gst + rr * D + c0) : make_float2(0.f, 0.f);
-                        px += gv[i].x;
-                        py += gv[i].y;
+                        gv[i] = rr < L ? f2_mul(*reinterpret_cast<const float2 *>(gst + rr * D + c0), l2e)
+                                       : make_float2(0.f, 0.f);
+                        ps = f2_add(ps, gv[i]);
                     }
                     // row-quarter sums of g per channel, [4][128] floats in the solve's scratch
                     float *gq = reinterpret_cast<float *>(sgen + PR_P);
-                    *reinterpret_cast<float2 *>(gq + tq * 128 + c0) = make_float2(px, py);
+                    *reinterpret_cast<float2 *>(gq + tq * 128 + c0) = ps;
                     if (named_bar_any(2, 256, *abort_flag != 0)) break;
                     float2 qs[4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) qs[q] = *reinterpret_cast<const float2 *>(gq + q * 128 + c0);
-                    const float gax = qs[0].x + qs[1].x, gay = qs[0].y + qs[1].y;   // G at the anchor row 31
-                    const float glx = gax + qs[2].x + qs[3].x, gly = gay + qs[2].y + qs[3].y;   // G at row 63
-                    float Gx = 0.f, Gy = 0.f;                                        // G before row r0
+                    const float2 ga = f2_add(qs[0], qs[1]);                  // G at the anchor row 31
+                    const float2 gl = f2_add(ga, f2_add(qs[2], qs[3]));      // G at row 63
+                    // Y = G - Ga, running over this thread's rows (starts at the row before r0)
+                    float2 Y = make_float2(-ga.x, -ga.y);
 #pragma unroll
                     for (int q = 0; q < 3; ++q)
-                        if (q < tq) {
-                            Gx += qs[q].x;
-                            Gy += qs[q].y;
-                        }
-                    const float ecx = ex2_approx(kLog2e * (glx - gax)), ecy = ex2_approx(kLog2e * (gly - gay));
+                        if (q < tq) Y = f2_add(Y, qs[q]);
+                    const float2 ec = make_float2(ex2_approx(gl.x - ga.x), ex2_approx(gl.y - ga.y));
                     // the channel pair is written as two rows; lanes 4-7 of every 8 write the odd
                     // channel first, so that one store instruction covers all eight swizzle phases
                     const bool odd_first = (lane >> 2) & 1;
@@ -901,34 +928,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         uint32_t hx[4], hy[4], qx4[4], qy4[4], cx[4], cy[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            float khx[2], khy[2], qhx[2], qhy[2], kcx[2], kcy[2], ktx[2], kty[2];
+                            float2 kh[2], qh[2], kc[2], kt[2];
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
                                 const int i = h8 * 8 + 2 * e + u, rr = r0 + i;
-                                Gx += gv[i].x;
-                                Gy += gv[i].y;
-                                const float yx = kLog2e * (Gx - gax), yy = kLog2e * (Gy - gay);
-                                const float epx = ex2_approx(yx), emx = ex2_approx(-yx);
-                                const float epy = ex2_approx(yy), emy = ex2_approx(-yy);
+                                Y = f2_add(Y, gv[i]);
+                                const float2 ep = make_float2(ex2_approx(Y.x), ex2_approx(Y.y));
+                                const float2 em = make_float2(ex2_approx(-Y.x), ex2_approx(-Y.y));
                                 const uint32_t kw = rr < L ? kst[rr * (D / 2) + cp] : 0u;
                                 const uint32_t qw = rr < L ? qst[rr * (D / 2) + cp] : 0u;
-                                khx[u] = lo_bf(kw) * epx;
-                                khy[u] = hi_bf(kw) * epy;
-                                qhx[u] = lo_bf(qw) * epx;
-                                qhy[u] = hi_bf(qw) * epy;
-                                kcx[u] = lo_bf(kw) * emx;
-                                kcy[u] = hi_bf(kw) * emy;
-                                ktx[u] = kcx[u] * ecx;
-                                kty[u] = kcy[u] * ecy;
+                                const float2 k2 = make_float2(lo_bf(kw), hi_bf(kw));
+                                const float2 q2 = make_float2(lo_bf(qw), hi_bf(qw));
+                                kh[u] = f2_mul(k2, ep);
+                                qh[u] = f2_mul(q2, ep);
+                                kc[u] = f2_mul(k2, em);
+                                kt[u] = f2_mul(kc[u], ec);
                             }
-                            hx[e] = pack_bf16(khx[0], khx[1]);
-                            hy[e] = pack_bf16(khy[0], khy[1]);
-                            qx4[e] = pack_bf16(qhx[0], qhx[1]);
-                            qy4[e] = pack_bf16(qhy[0], qhy[1]);
-                            cx[e] = pack_bf16(kcx[0], kcx[1]);
-                            cy[e] = pack_bf16(kcy[0], kcy[1]);
-                            ktr[h8 * 4 + e] = pack_f16(ktx[0], ktx[1]);
-                            ktr[8 + h8 * 4 + e] = pack_f16(kty[0], kty[1]);
+                            hx[e] = pack_bf16(kh[0].x, kh[1].x);
+                            hy[e] = pack_bf16(kh[0].y, kh[1].y);
+                            qx4[e] = pack_bf16(qh[0].x, qh[1].x);
+                            qy4[e] = pack_bf16(qh[0].y, qh[1].y);
+                            cx[e] = pack_bf16(kc[0].x, kc[1].x);
+                            cy[e] = pack_bf16(kc[0].y, kc[1].y);
+                            ktr[h8 * 4 + e] = pack_f16(kt[0].x, kt[1].x);
+                            ktr[8 + h8 * 4 + e] = pack_f16(kt[0].y, kt[1].y);
                         }
                         const int j = 2 * tq + h8;   // 16-byte chunk (8 tokens) of a channel row
                         const uint32_t ra = c0 + (odd_first ? 1 : 0), rb2 = c0 + (odd_first ? 0 : 1);
@@ -936,18 +959,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         for (int tile = 0; tile < 3; ++tile) {
                             const uint32_t base = sbase + (tile == 0 ? PR_KH : (tile == 1 ? PR_QH : PR_KC));
                             const uint32_t *X = tile == 0 ? hx : (tile == 1 ? qx4 : cx);
-                            const uint32_t *Y = tile == 0 ? hy : (tile == 1 ? qy4 : cy);
-                            st_shared_v4(base + sw128(ra, j), odd_first ? Y[0] : X[0], odd_first ? Y[1] : X[1],
-                                         odd_first ? Y[2] : X[2], odd_first ? Y[3] : X[3]);
-                            st_shared_v4(base + sw128(rb2, j), odd_first ? X[0] : Y[0], odd_first ? X[1] : Y[1],
-                                         odd_first ? X[2] : Y[2], odd_first ? X[3] : Y[3]);
+                            const uint32_t *Yw = tile == 0 ? hy : (tile == 1 ? qy4 : cy);
+                            st_shared_v4(base + sw128(ra, j), odd_first ? Yw[0] : X[0], odd_first ? Yw[1] : X[1],
+                                         odd_first ? Yw[2] : X[2], odd_first ? Yw[3] : X[3]);
+                            st_shared_v4(base + sw128(rb2, j), odd_first ? X[0] : Yw[0], odd_first ? X[1] : Yw[1],
+                                         odd_first ? X[2] : Yw[2], odd_first ? X[3] : Yw[3]);
                         }
                     }
                     if (tq == 0) {
                         *reinterpret_cast<float2 *>(dec_all + (kk & 1) * 128 + c0) =
-                            make_float2(ex2_approx(kLog2e * glx), ex2_approx(kLog2e * gly));
-                        *reinterpret_cast<float2 *>(ega_s + c0) =
-                            make_float2(ex2_approx(kLog2e * gax), ex2_approx(kLog2e * gay));
+                            make_float2(ex2_approx(gl.x), ex2_approx(gl.y));
+                        *reinterpret_cast<float2 *>(ega_s + c0) = make_float2(ex2_approx(ga.x), ex2_approx(ga.y));
                     }
                 }
                 fence_proxy_async_smem();
@@ -973,8 +995,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     st_shared_v4(a, pack_f16(lo_bf(x.x), hi_bf(x.x)), pack_f16(lo_bf(x.y), hi_bf(x.y)),
                                  pack_f16(lo_bf(x.z), hi_bf(x.z)), pack_f16(lo_bf(x.w), hi_bf(x.w)));
                 }
-                fence_proxy_async_smem();
-
                 // -------- S2 epilogue: A (fp32, masked, beta-scaled) and Aqk (fp16 + bf16); Kt^T out
                 // (part C of the previous set, over A / T and the AV operand, must be read out)
                 if (kk >= 1) wait_bar(BAR(PB_OUTC_FREE), (kk - 1) & 1, abort_flag);
@@ -997,6 +1017,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     uint32_t a[32];
                     tmem_ld32(tmem + lane_base + COL_P1 + half * 32, a);
                     tmem_wait_ld();
+                    if (t == 0) KDA_TRACE_POINT(m, 27);
                     if (lrow < 64) {
                         const int rr = lrow;
                         const float br = beta_s[rr];
@@ -1030,7 +1051,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     float *T = wsf + PR_T / 4;
                     T[(t >> 4) * AKK_LD + 16 + (t & 15)] = 0.f;               // rows 0-15, cols 16-31
                     T[(32 + (t >> 4)) * AKK_LD + 48 + (t & 15)] = 0.f;        // rows 32-47, cols 48-63
+                    // S3 (a): the four 16 x 16 diagonal blocks of T = (I + A)^-1. Warp 4 has just
+                    // written blocks 0 and 1 of A, warp 9 blocks 2 and 3; each lane solves one column
+                    // of its block by forward substitution, right-looking: once x[j] is final it is
+                    // folded into every later row, so a row costs one FMA on the dependent path.
+                    if (warp == 4 || warp == 9) {
+                        __syncwarp();
+                        const int wb = (warp == 4 ? 0 : 2) + (lane >> 4), li = lane & 15;
+                        const float *Ab = wsf + PR_AKK / 4 + 16 * wb * AKK_LD + 16 * wb;
+                        float x[16];
+#pragma unroll
+                        for (int r = 0; r < 16; ++r) x[r] = r == li ? 1.f : 0.f;
+#pragma unroll
+                        for (int j = 0; j < 15; ++j)
+#pragma unroll
+                            for (int r = j + 1; r < 16; ++r) x[r] = fmaf(-Ab[r * AKK_LD + j], x[j], x[r]);
+#pragma unroll
+                        for (int r = 0; r < 16; ++r) T[(16 * wb + r) * AKK_LD + 16 * wb + li] = x[r];
+                    }
                 }
+                if (t == 0) KDA_TRACE_POINT(m, 28);
                 fence_proxy_async_smem();
                 tc_fence_before();
                 if (named_bar_any(2, 256, *abort_flag != 0)) break;
@@ -1040,7 +1080,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
 
                 // -------- S3: T = (I + A)^-1 by recursive blocking:
-                //   (a) the four 16 x 16 diagonal blocks by forward substitution,
+                //   (a) the four 16 x 16 diagonal blocks by forward substitution (done above, in the
+                //       S2 epilogue, by the warps that wrote those blocks of A),
                 //   (b) the two 16 x 16 blocks below them inside each 32 x 32 diagonal block,
                 //   (c) the 32 x 32 block below the diagonal,
                 // each off-diagonal block as  T_IJ = -T_II (A_IJ T_JJ).
@@ -1048,31 +1089,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const float *A = wsf + PR_AKK / 4;
                     float *T = wsf + PR_T / 4;
                     float *P = wsf + PR_P / 4;
-                    if (t < 128) {
-                        const int wb = t >> 5, li = t & 31;
-                        if (li < 16) {
-                            // column li of the inverse of diagonal block wb, row by row; the block's
-                            // rows of A are read as float4 (entries on and above the diagonal are 0)
-                            float x[16];
-#pragma unroll
-                            for (int rr = 0; rr < 16; ++rr) {
-                                const float *arow = A + (16 * wb + rr) * AKK_LD + 16 * wb;
-                                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-                                for (int j4 = 0; j4 < (rr + 3) / 4; ++j4) {
-                                    const float4 av = *reinterpret_cast<const float4 *>(arow + 4 * j4);
-                                    if (4 * j4 + 0 < rr) a0 = fmaf(av.x, x[4 * j4 + 0], a0);
-                                    if (4 * j4 + 1 < rr) a1 = fmaf(av.y, x[4 * j4 + 1], a1);
-                                    if (4 * j4 + 2 < rr) a2 = fmaf(av.z, x[4 * j4 + 2], a2);
-                                    if (4 * j4 + 3 < rr) a3 = fmaf(av.w, x[4 * j4 + 3], a3);
-                                }
-                                x[rr] = ((rr == li) ? 1.f : 0.f) - ((a0 + a1) + (a2 + a3));
-                            }
-#pragma unroll
-                            for (int rr = 0; rr < 16; ++rr) T[(16 * wb + rr) * AKK_LD + 16 * wb + li] = x[rr];
-                        }
-                    }
-                    if (named_bar_any(2, 256, *abort_flag != 0)) break;
                     if (t == 0) KDA_TRACE_POINT(m, 10);
                     // T' = T diag(beta) is written straight into its two operand tiles as each block of
                     // T becomes final: fp16 (rows 0..63 of the [T'; Aqk] tile) and bf16 (TB); the blocks
@@ -1111,6 +1127,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             st_shared_v2(tp_addr(sbase + PR_TB, r, c), pack_bf16(x0, x1), pack_bf16(x2, x3));
                         }
                         if (named_bar_any(2, 256, *abort_flag != 0)) break;
+                        if (t == 0) KDA_TRACE_POINT(m, 29);
                         const float *trow = T + (16 * I + rr) * AKK_LD + 16 * I;
                         p0 = 0.f;
                         p1 = 0.f;
@@ -1130,6 +1147,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const float x0 = -p0 * beta_s[c], x1 = -p1 * beta_s[c + 1];
                         st_shared_u32(tp_addr(sbase + PR_AVT, r, c), pack_f16(x0, x1));
                         st_shared_u32(tp_addr(sbase + PR_TB, r, c), pack_bf16(x0, x1));
+                        if (t == 0) KDA_TRACE_POINT(m, 13);
                     }
                     if (named_bar_any(2, 256, *abort_flag != 0)) break;
                     if (t == 0) KDA_TRACE_POINT(m, 11);
@@ -1159,6 +1177,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         *reinterpret_cast<float4 *>(P + rr * 32 + (((c4 >> 2) ^ (rr & 7)) << 2)) =
                             make_float4(p0, p1, p2, p3);
                         if (named_bar_any(2, 256, *abort_flag != 0)) break;
+                        if (t == 0) KDA_TRACE_POINT(m, 14);
                         const float *trow = T + (32 + rr) * AKK_LD + 32;
                         p0 = p1 = p2 = p3 = 0.f;
 #pragma unroll
