@@ -1155,6 +1155,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     // Lane = row, warp = 4-column group, so the T and P2 reads are warp-uniform
                     // (broadcast) and the zero block T[0:16, 16:32] is skipped by whole warps. P2 is
                     // stored with its 16-byte groups XOR-swizzled by row to keep the stores conflict-free.
+                    // A warp reads back only the P2 columns it wrote, so it waits for no other warp.
                     {
                         const int rr = t & 31, c4 = (t >> 5) * 4;
                         const float *arow = A + (32 + rr) * AKK_LD;
@@ -1176,7 +1177,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         }
                         *reinterpret_cast<float4 *>(P + rr * 32 + (((c4 >> 2) ^ (rr & 7)) << 2)) =
                             make_float4(p0, p1, p2, p3);
-                        if (named_bar_any(2, 256, *abort_flag != 0)) break;
+                        __syncwarp();
                         if (t == 0) KDA_TRACE_POINT(m, 14);
                         const float *trow = T + (32 + rr) * AKK_LD + 32;
                         p0 = p1 = p2 = p3 = 0.f;
