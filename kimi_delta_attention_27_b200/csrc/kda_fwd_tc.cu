@@ -866,12 +866,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #endif
                 const int m = static_cast<int>(chunkq[kk & 3]);   // this CTA's kk-th chunk
                 const bool no_chunk = m >= nch;
+                if (!no_chunk) {
+                    // partial chunk: the staged rows past the sequence's end hold the next
+                    // sequence's tokens (or TMA fill); zero them so that S1 needs no row masks
+                    const int64_t tz = bos + static_cast<int64_t>(m) * C;
+                    const int Lz = static_cast<int>(eos - tz < C ? eos - tz : C);
+                    if (Lz < C) {
+                        for (int e = t; e < (C - Lz) * 16; e += 256) {
+                            const uint32_t off = static_cast<uint32_t>((Lz + (e >> 4)) * 256 + (e & 15) * 16);
+                            st_shared_v4(sbase + PR_STG + STG_Q + off, 0u, 0u, 0u, 0u);
+                            st_shared_v4(sbase + PR_STG + STG_K + off, 0u, 0u, 0u, 0u);
+                        }
+                        for (int e = t; e < (C - Lz) * 32; e += 256)
+                            st_shared_v4(sbase + PR_STG + STG_G + static_cast<uint32_t>((Lz + (e >> 5)) * 512 + (e & 31) * 16),
+                                         0u, 0u, 0u, 0u);
+                    }
+                }
                 if (named_bar_any(2, 256, no_chunk || *abort_flag != 0)) {
                     if (t == 0) mbar_arrive(BAR(PB_OUTA_READY));   // the publisher's end signal
                     break;
                 }
-                const int64_t t0 = bos + static_cast<int64_t>(m) * C;
-                const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
                 const float *beta_s = reinterpret_cast<const float *>(miscg + M_BETAQ) + (kk & 1) * C;
 #ifdef KDA_TRACE
                 if (t == 0 && blockIdx.x / 4 == KDA_TRACE_CLUSTER_ID && m < 64) {
@@ -884,59 +898,65 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
                 // -------- S1: running log-decay and the anchored factors. A thread owns a pair of
                 // adjacent channels (c0, c0 + 1) over one quarter of the rows (16 tokens), so q and k
-                // are read as bf16 pairs and g as float pairs.
-                uint32_t ktr[16];   // Kt^T of this thread: 4 fp16 pairs x 2 chunks x 2 channels
+                // are read as bf16 pairs and g as float pairs. It takes its rows in two passes of 8;
+                // lanes 4-7 of every 8 take the two halves in the other order, so that each store
+                // instruction covers all eight swizzle phases. Rows past the end of a partial chunk
+                // were zeroed above.
+                uint32_t ktr[16];   // Kt^T of this thread: 4 fp16 pairs x 2 passes x 2 channels
+                const bool flip = (lane >> 2) & 1;
                 {
                     const int grp = (warp - 4) & 3;
                     const int cp = grp * 16 + (lane & 15);
                     const int tq = 2 * ((warp - 4) >> 2) + (lane >> 4);
                     const int c0 = 2 * cp, r0 = 16 * tq;
+                    const int rp0 = r0 + (flip ? 8 : 0), rp1 = r0 + (flip ? 0 : 8);   // first row of each pass
                     const float *gst = reinterpret_cast<const float *>(sgen + PR_STG + STG_G);
                     const uint32_t *qst = reinterpret_cast<const uint32_t *>(sgen + PR_STG + STG_Q);
                     const uint32_t *kst = reinterpret_cast<const uint32_t *>(sgen + PR_STG + STG_K);
-                    // g of the channel pair in log2 units (x, y = channels c0, c0 + 1)
+                    // g of the channel pair in log2 units (x, y = channels c0, c0 + 1), in pass order
                     const float2 l2e = make_float2(kLog2e, kLog2e);
                     float2 gv[16];
-                    float2 ps = make_float2(0.f, 0.f);
+                    float2 sp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const int rr = r0 + i;
-                        gv[i] = rr < L ? f2_mul(*reinterpret_cast<const float2 *>(gst + rr * D + c0), l2e)
-                                       : make_float2(0.f, 0.f);
-                        ps = f2_add(ps, gv[i]);
+                        const int rr = (i < 8 ? rp0 : rp1) + (i & 7);
+                        gv[i] = f2_mul(*reinterpret_cast<const float2 *>(gst + rr * D + c0), l2e);
+                        sp[i >> 3] = f2_add(sp[i >> 3], gv[i]);
                     }
                     // row-quarter sums of g per channel, [4][128] floats in the solve's scratch
                     float *gq = reinterpret_cast<float *>(sgen + PR_P);
-                    *reinterpret_cast<float2 *>(gq + tq * 128 + c0) = ps;
+                    *reinterpret_cast<float2 *>(gq + tq * 128 + c0) = f2_add(sp[0], sp[1]);
                     if (named_bar_any(2, 256, *abort_flag != 0)) break;
                     float2 qs[4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) qs[q] = *reinterpret_cast<const float2 *>(gq + q * 128 + c0);
                     const float2 ga = f2_add(qs[0], qs[1]);                  // G at the anchor row 31
                     const float2 gl = f2_add(ga, f2_add(qs[2], qs[3]));      // G at row 63
-                    // Y = G - Ga, running over this thread's rows (starts at the row before r0)
-                    float2 Y = make_float2(-ga.x, -ga.y);
+                    // Y = G - Ga, running over a pass's rows; Y0 is its value before row r0
+                    float2 Y0 = make_float2(-ga.x, -ga.y);
 #pragma unroll
                     for (int q = 0; q < 3; ++q)
-                        if (q < tq) Y = f2_add(Y, qs[q]);
+                        if (q < tq) Y0 = f2_add(Y0, qs[q]);
                     const float2 ec = make_float2(ex2_approx(gl.x - ga.x), ex2_approx(gl.y - ga.y));
-                    // the channel pair is written as two rows; lanes 4-7 of every 8 write the odd
-                    // channel first, so that one store instruction covers all eight swizzle phases
-                    const bool odd_first = (lane >> 2) & 1;
+                    // pass 0 starts after the rows of the lower half when it is the upper half
+                    const float2 y1 = f2_add(Y0, sp[1]);
+                    float2 Y = flip ? y1 : Y0;
 #pragma unroll
-                    for (int h8 = 0; h8 < 2; ++h8) {
+                    for (int ps = 0; ps < 2; ++ps) {
+                        if (ps == 1) Y = flip ? Y0 : Y;
+                        const int rb = ps == 0 ? rp0 : rp1;
                         uint32_t hx[4], hy[4], qx4[4], qy4[4], cx[4], cy[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             float2 kh[2], qh[2], kc[2], kt[2];
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
-                                const int i = h8 * 8 + 2 * e + u, rr = r0 + i;
+                                const int i = ps * 8 + 2 * e + u, rr = rb + 2 * e + u;
                                 Y = f2_add(Y, gv[i]);
                                 const float2 ep = make_float2(ex2_approx(Y.x), ex2_approx(Y.y));
                                 const float2 em = make_float2(ex2_approx(-Y.x), ex2_approx(-Y.y));
-                                const uint32_t kw = rr < L ? kst[rr * (D / 2) + cp] : 0u;
-                                const uint32_t qw = rr < L ? qst[rr * (D / 2) + cp] : 0u;
+                                const uint32_t kw = kst[rr * (D / 2) + cp];
+                                const uint32_t qw = qst[rr * (D / 2) + cp];
                                 const float2 k2 = make_float2(lo_bf(kw), hi_bf(kw));
                                 const float2 q2 = make_float2(lo_bf(qw), hi_bf(qw));
                                 kh[u] = f2_mul(k2, ep);
@@ -950,20 +970,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             qy4[e] = pack_bf16(qh[0].y, qh[1].y);
                             cx[e] = pack_bf16(kc[0].x, kc[1].x);
                             cy[e] = pack_bf16(kc[0].y, kc[1].y);
-                            ktr[h8 * 4 + e] = pack_f16(kt[0].x, kt[1].x);
-                            ktr[8 + h8 * 4 + e] = pack_f16(kt[0].y, kt[1].y);
+                            ktr[ps * 4 + e] = pack_f16(kt[0].x, kt[1].x);
+                            ktr[8 + ps * 4 + e] = pack_f16(kt[0].y, kt[1].y);
                         }
-                        const int j = 2 * tq + h8;   // 16-byte chunk (8 tokens) of a channel row
-                        const uint32_t ra = c0 + (odd_first ? 1 : 0), rb2 = c0 + (odd_first ? 0 : 1);
+                        const int j = (rb >> 3);   // 16-byte chunk (8 tokens) of a channel row
 #pragma unroll
                         for (int tile = 0; tile < 3; ++tile) {
                             const uint32_t base = sbase + (tile == 0 ? PR_KH : (tile == 1 ? PR_QH : PR_KC));
                             const uint32_t *X = tile == 0 ? hx : (tile == 1 ? qx4 : cx);
                             const uint32_t *Yw = tile == 0 ? hy : (tile == 1 ? qy4 : cy);
-                            st_shared_v4(base + sw128(ra, j), odd_first ? Yw[0] : X[0], odd_first ? Yw[1] : X[1],
-                                         odd_first ? Yw[2] : X[2], odd_first ? Yw[3] : X[3]);
-                            st_shared_v4(base + sw128(rb2, j), odd_first ? X[0] : Yw[0], odd_first ? X[1] : Yw[1],
-                                         odd_first ? X[2] : Yw[2], odd_first ? X[3] : Yw[3]);
+                            st_shared_v4(base + sw128(c0, j), X[0], X[1], X[2], X[3]);
+                            st_shared_v4(base + sw128(c0 + 1, j), Yw[0], Yw[1], Yw[2], Yw[3]);
                         }
                     }
                     if (tq == 0) {
@@ -1010,8 +1027,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                             for (int h8 = 0; h8 < 2; ++h8) {
                                 const uint32_t *w4 = ktr + ch * 8 + h8 * 4;
-                                st_shared_v4(sbase + PR_KC + sw128(2 * cp + ch, 2 * tq + h8), w4[0], w4[1], w4[2],
-                                             w4[3]);
+                                st_shared_v4(sbase + PR_KC + sw128(2 * cp + ch, 2 * tq + (h8 ^ (flip ? 1 : 0))), w4[0],
+                                             w4[1], w4[2], w4[3]);
                             }
                     }
                     uint32_t a[32];
