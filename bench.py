@@ -270,8 +270,13 @@ def main():
                     help="tokens (all heads) per reference-arm step")
     ap.add_argument("--e2e-slice", type=int, default=1 << 16,
                     help="tokens per host->device slice in the end-to-end measurement")
+    ap.add_argument("--decode", default=None, metavar="BxH[:bf16]",
+                    help="time the single-token decode step instead (e.g. 256x32 or 256x32:bf16); "
+                         "prints its own line, not the prefill metric")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.decode:
+        return decode_main(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -301,12 +306,7 @@ def main():
         step()
     torch.cuda.synchronize()
 
-    sampler = None
-    if rank == 0:
-        props = torch.cuda.get_device_properties(torch.cuda.current_device())
-        uuid = str(getattr(props, "uuid", ""))
-        sampler = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else
-                               (uuid or torch.cuda.current_device()))
+    sampler = current_gpu_sampler() if rank == 0 else None
     if sampler:
         sampler.start()
         time.sleep(0.3)
@@ -382,6 +382,85 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+    return 0
+
+
+def current_gpu_sampler():
+    """A ClockSampler for this process's GPU, named by UUID so that nvidia-smi's
+    numbering cannot pick another GPU."""
+    import torch
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    uuid = str(getattr(props, "uuid", ""))
+    return ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else
+                        (uuid or torch.cuda.current_device()))
+
+
+def decode_main(args):
+    """The decode step (kda_decode) on one GPU: B requests x H heads, one token per
+    request per step, states updated in place. Bound by HBM: each (request, head)
+    reads and writes its 128 x 128 state."""
+    import torch
+    import kimi_delta_attention_27_b200 as kda
+    from kimi_delta_attention_27_b200.inputs import make_inputs
+    spec, _, sdt = args.decode.partition(":")
+    B, H = (int(x) for x in spec.lower().split("x"))
+    sdt = sdt or "fp32"
+    steps = args.steps
+    # one token per request per step; inputs for all timed and warm-up steps are made up front
+    nstep = args.warmup + steps
+    inp = make_inputs({"B": B, "T": nstep, "H": H, "lengths": None, "g_mu": 3.0, "init": sdt,
+                       "final": sdt, "seed": 90}, device="cuda")
+    toks = [tuple(inp[n][:, t].contiguous() for n in ("q", "k", "v", "g", "beta")) for t in range(nstep)]
+    S = inp["h0"]
+    out = torch.empty((B, H, D), dtype=torch.bfloat16, device="cuda")
+    del inp
+    stream = torch.cuda.current_stream()
+
+    def step(t):
+        q, k, v, g, beta = toks[t]
+        kda.kda_decode(q, k, v, g, beta, state_in=S, state_out=S, out=out)
+
+    for t in range(args.warmup):
+        step(t)
+    torch.cuda.synchronize()
+    sampler = current_gpu_sampler()
+    sampler.start()
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True); t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("timed")
+    t0.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        step(args.warmup + i)
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
+    clocks = sampler.stop()
+    ms_per_step = t0.elapsed_time(t1) / steps
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    esz = 4 if sdt == "fp32" else 2
+    # per (request, head): the state read and written, q, k, v, out (bf16), g (fp32), beta
+    unit_bytes = 2 * D * D * esz + 4 * D * 2 + D * 4 + 4
+    alg_bytes = B * H * unit_bytes
+    peaks = load_peaks()
+    achieved = alg_bytes / (launch_ms / 1e3) / 1e9
+    line = {
+        "metric": "KDA decode step tokens/s (one token per request, all heads)", "value": B / (ms_per_step / 1e3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "dtype": "f32" if sdt == "fp32" else "bf16", "data": "synthetic",
+        "config": {"workload": f"decode step: {B} requests x {H} heads, {sdt} states updated in place",
+                   "requests": B, "heads": H, "state_dtype": sdt,
+                   "l2": "states larger than L2 (no flush needed)" if alg_bytes > 126e6 else "states fit in L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
+                     "kernel": f"kda_decode_kernel<{'true' if sdt == 'fp32' else 'false'}>",
+                     "alg_bytes_per_launch": alg_bytes, "bytes_per_unit": unit_bytes, "avg_launch_ms": launch_ms},
+        "gpu_launches": steps, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
     return 0
 
 

@@ -1,9 +1,9 @@
 /*
  * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention forward library.
  *
- * One operation: the chunkwise forward (prefill) pass of Kimi Delta Attention,
- * i.e. for every sequence and head the recurrence of the Kimi Linear feature
- * page (chapter 4, "innovation 2", state-update equation)
+ * The chunkwise forward (prefill) pass of Kimi Delta Attention, i.e. for every
+ * sequence and head the recurrence of the Kimi Linear feature page (chapter 4,
+ * "innovation 2", state-update equation)
  *
  *     S_t = (Diag(alpha_t) - beta_t k_t (k_t (.) alpha_t)^T) S_{t-1} + beta_t k_t v_t^T
  *     o_t = scale * S_t^T q_t,          alpha_t = exp(g_t) per key channel,
@@ -14,7 +14,8 @@
  * constraints"): query, key, value, gate, beta tensors, head dims K = V = 128
  * only, variable-length packing through cu_seqlens with batch 1, and optional
  * bf16 or fp32 initial / final states whose dtypes must match when both are
- * given.
+ * given. A single-token step of the same recurrence for a batch of requests
+ * (decode) is kda_decode.
  *
  * Conventions for every entry point below:
  *  - All tensor pointers are DEVICE pointers on the current CUDA device, owned
@@ -51,7 +52,8 @@ typedef enum {
     KDA_ERR_BAD_ALIGNMENT = 7,     /* a tensor pointer is not 16-byte aligned            */
     KDA_ERR_TOO_LARGE = 8,         /* sizes exceed what the library indexes              */
     KDA_ERR_TIMEOUT = 9,           /* a kernel gave up on a bounded wait (see kda_device_error) */
-    KDA_ERR_NOALLOC_LIMIT = 10     /* kda_fwd_noalloc: more (sequence, head) pairs than its scratch holds */
+    KDA_ERR_NOALLOC_LIMIT = 10,    /* kda_fwd_noalloc: more (sequence, head) pairs than its scratch holds */
+    KDA_ERR_STATE_OVERLAP = 11     /* kda_decode: distinct state_in and state_out buffers overlap */
 } kda_status;
 
 typedef enum { KDA_DTYPE_NONE = 0, KDA_DTYPE_BF16 = 1, KDA_DTYPE_FP32 = 2 } kda_dtype;
@@ -137,6 +139,40 @@ kda_status kda_fwd_noalloc(const void *q, const void *k, const void *v, const fl
                            int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
                            kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype,
                            void *out, kda_stream_t stream);
+
+/*
+ * kda_decode -- one recurrent step (a single new token) for a batch of
+ * independent requests, each with its own state per head.
+ *
+ * For every request b and head h this is the state-update equation above for
+ * one token, with the output read from the updated state (as in kda_fwd):
+ *     S <- (Diag(alpha) - beta k (k (.) alpha)^T) S + beta k v^T,   o = scale * S^T q,
+ * alpha = exp(g) per key channel. kda_fwd over a sequence of length 1 with an
+ * initial and a final state computes the same thing; this entry point exists
+ * because a decode step is bound by reading and writing the 128 x 128 state,
+ * which it does once, with no chunk machinery. The pages describe the step (the
+ * decode-speed claims of the Kimi Linear feature page) but define no such call.
+ *
+ * Layouts (row-major, innermost last, all contiguous):
+ *   q, k, v  : bf16 [batch, num_heads, 128]
+ *   g        : fp32 [batch, num_heads, 128]  log alpha (raw, no activation)
+ *   beta     : fp32 [batch, num_heads]
+ *   out      : bf16 [batch, num_heads, 128]  (written)
+ *   state_in, state_out : [batch, num_heads, 128 (key), 128 (value)], value
+ *              index fastest, dtype state_dtype (KDA_DTYPE_BF16 or _FP32).
+ *   state_in  == NULL means zero states; state_out == NULL means the updated
+ *   states are not written. state_out may be the same pointer as state_in (the
+ *   step then updates the states in place); distinct buffers that overlap are
+ *   refused with KDA_ERR_STATE_OVERLAP.
+ * The state is carried in fp32 inside the step; a bf16 state is rounded to
+ * nearest even when written. head_dim_k and head_dim_v must both be 128; all
+ * tensor pointers must be 16-byte aligned (beta 4-byte). batch == 0 is a no-op.
+ * Nothing is allocated. Returns KDA_OK once the work is enqueued.
+ */
+kda_status kda_decode(const void *q, const void *k, const void *v, const float *g,
+                      const float *beta, float scale, int32_t batch, int32_t num_heads,
+                      int32_t head_dim_k, int32_t head_dim_v, const void *state_in,
+                      void *state_out, kda_dtype state_dtype, void *out, kda_stream_t stream);
 
 /*
  * kda_device_error -- synchronise the current device, then read and clear the

@@ -1,4 +1,4 @@
-"""B200 (sm_100a) Kimi Delta Attention forward library: Python binding.
+"""B200 (sm_100a) Kimi Delta Attention library (prefill forward and decode step): Python binding.
 
 The work happens in ``libkda.so`` (hand-written CUDA kernels behind the C ABI
 declared in ``include/kda.h``). This module only marshals torch tensors into
@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libkda.so")
 
 # entry points declared in include/kda.h
-EXPORTS = ("kda_device_error", "kda_fwd", "kda_fwd_noalloc", "kda_status_string", "kda_version")
+EXPORTS = ("kda_decode", "kda_device_error", "kda_fwd", "kda_fwd_noalloc", "kda_status_string", "kda_version")
 
 # (sequence, head) pairs per kda_fwd_noalloc call (KDA_NOALLOC_MAX_UNITS in include/kda.h)
 NOALLOC_MAX_UNITS = 32
@@ -52,6 +52,8 @@ def load_library(path: str | None = None):
         for name in ("kda_fwd", "kda_fwd_noalloc"):
             getattr(lib, name).restype = ctypes.c_int
             getattr(lib, name).argtypes = fwd_args
+        lib.kda_decode.restype = ctypes.c_int
+        lib.kda_decode.argtypes = [P, P, P, P, P, ctypes.c_float, i32, i32, i32, i32, P, P, ctypes.c_int, P, P]
         lib.kda_status_string.restype = ctypes.c_char_p
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_version.restype = ctypes.c_int32
@@ -174,3 +176,50 @@ def _fwd(entry, q, k, v, g, beta, scale, cu_seqlens, initial_state, final_state,
     if st != 0:
         raise KdaError(st, lib.kda_status_string(st).decode())
     return out, final_state
+
+
+def kda_decode(q, k, v, g, beta, state_in=None, state_out=None, scale: float | None = None, out=None,
+               state_dtype=None, stream=None):
+    """One recurrent step for a batch of requests (see include/kda.h, kda_decode).
+
+    q, k, v: bf16 [B, H, 128]; g: fp32 [B, H, 128] (raw log alpha); beta: fp32 [B, H];
+    state_in: [B, H, 128, 128] bf16/fp32 or None (zero states). ``state_out`` may be
+    ``state_in`` itself (update in place) or a separate buffer; if it is None and
+    ``state_dtype`` is given, one is allocated. ``out`` may be passed preallocated.
+    Returns (out, state_out or None).
+    """
+    import torch
+    _check("q", q, torch.bfloat16, 3)
+    _check("k", k, torch.bfloat16, 3)
+    _check("v", v, torch.bfloat16, 3)
+    _check("g", g, torch.float32, 3)
+    _check("beta", beta, torch.float32, 2)
+    B, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if k.shape != q.shape or g.shape != q.shape or v.shape[:2] != q.shape[:2] or beta.shape != (B, H):
+        raise ValueError("q/k/g must share [B, H, 128]; v [B, H, 128]; beta [B, H]")
+    if state_in is not None:
+        _check("state_in", state_in, None, 4)
+    if state_out is None and state_dtype is not None:
+        state_out = torch.empty((B, H, Dk, Dv), dtype=state_dtype, device=q.device)
+    if state_out is not None:
+        _check("state_out", state_out, None, 4)
+    if state_in is not None and state_out is not None and state_in.dtype != state_out.dtype:
+        raise ValueError("state_in and state_out must have the same dtype")
+    st_t = state_in if state_in is not None else state_out
+    code = _dtype_code(st_t)
+    if out is None:
+        out = torch.empty((B, H, Dv), dtype=torch.bfloat16, device=q.device)
+    else:
+        _check("out", out, torch.bfloat16, 3)
+    if scale is None:
+        scale = Dk ** -0.5
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    lib = load_library()
+    st = lib.kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), int(B), int(H),
+                        int(Dk), int(Dv), _ptr(state_in), _ptr(state_out), code if code >= 0 else 99,
+                        _ptr(out), ctypes.c_void_p(int(stream)))
+    if st != 0:
+        raise KdaError(st, lib.kda_status_string(st).decode())
+    return out, state_out

@@ -92,11 +92,13 @@ const char *kda_status_string(kda_status s) {
         case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a kernel gave up waiting on a barrier and stopped";
         case KDA_ERR_NOALLOC_LIMIT:
             return "KDA_ERR_NOALLOC_LIMIT: kda_fwd_noalloc takes at most 32 (sequence, head) pairs per call";
+        case KDA_ERR_STATE_OVERLAP:
+            return "KDA_ERR_STATE_OVERLAP: kda_decode state_in and state_out overlap without being the same buffer";
     }
     return "KDA_ERR_UNKNOWN";
 }
 
-int32_t kda_version(void) { return (1 << 16) | 1; }
+int32_t kda_version(void) { return (1 << 16) | 2; }
 
 kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
                    const float *beta, float scale, const int32_t *cu_seqlens,
@@ -127,6 +129,45 @@ kda_status kda_fwd_noalloc(const void *q, const void *k, const void *v, const fl
                                   final_dtype, out, true, &p, &rows);
     if (st != KDA_OK || p.num_seqs == 0) return st;
     const cudaError_t err = kda::launch_fwd_tc_noalloc(p, rows, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode(const void *q, const void *k, const void *v, const float *g,
+                      const float *beta, float scale, int32_t batch, int32_t num_heads,
+                      int32_t head_dim_k, int32_t head_dim_v, const void *state_in,
+                      void *state_out, kda_dtype state_dtype, void *out, kda_stream_t stream) {
+    if (head_dim_k != kda::kHeadDim || head_dim_v != kda::kHeadDim) return KDA_ERR_BAD_SHAPE;
+    if (batch < 0 || num_heads < 1) return KDA_ERR_BAD_SHAPE;
+    if ((state_in || state_out) && state_dtype != KDA_DTYPE_BF16 && state_dtype != KDA_DTYPE_FP32)
+        return KDA_ERR_STATE_DTYPE;
+    const int64_t units = static_cast<int64_t>(batch) * num_heads;
+    if (units > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL_PTR;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(out) ||
+        !aligned16(state_in) || !aligned16(state_out) || (reinterpret_cast<uintptr_t>(beta) & 3u))
+        return KDA_ERR_BAD_ALIGNMENT;
+    if (units > 0x7fffffffLL) return KDA_ERR_TOO_LARGE;
+    if (state_in && state_out && state_in != state_out) {
+        // distinct state buffers must not overlap
+        const uintptr_t a = reinterpret_cast<uintptr_t>(state_in), b = reinterpret_cast<uintptr_t>(state_out);
+        const uintptr_t bytes = static_cast<uintptr_t>(units) * kda::kHeadDim * kda::kHeadDim *
+                                (state_dtype == KDA_DTYPE_FP32 ? 4u : 2u);
+        if (a < b + bytes && b < a + bytes) return KDA_ERR_STATE_OVERLAP;
+    }
+    if (units == 0) return KDA_OK;
+    int qerr = 0;
+    if (!device_is_sm100(&qerr)) return qerr ? KDA_ERR_CUDA : KDA_ERR_UNSUPPORTED_DEVICE;
+    kda::DecodeParams p;
+    p.q = static_cast<const uint16_t *>(q);
+    p.k = static_cast<const uint16_t *>(k);
+    p.v = static_cast<const uint16_t *>(v);
+    p.g = g;
+    p.beta = beta;
+    p.scale = scale;
+    p.state_in = state_in;
+    p.state_out = state_out;
+    p.state_fp32 = state_dtype == KDA_DTYPE_FP32;
+    p.out = static_cast<uint16_t *>(out);
+    const cudaError_t err = kda::launch_decode(p, units, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

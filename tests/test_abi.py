@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for st in range(0, 11):
+    for st in range(0, 12):
         s = kda.status_string(st)
         assert s.startswith("KDA_"), s
     assert kda.status_string(1234) == "KDA_ERR_UNKNOWN"
