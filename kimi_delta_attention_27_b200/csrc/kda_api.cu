@@ -3,6 +3,7 @@
 
 #include "../../include/kda.h"
 #include "kda_internal.h"
+#include "kda_decode.h"
 
 static_assert(kda::kNoAllocMaxUnits == KDA_NOALLOC_MAX_UNITS, "scratch limit of kda_fwd_noalloc");
 

@@ -21,6 +21,7 @@
 #include <cuda_runtime.h>
 
 #include "kda_internal.h"
+#include "kda_decode.h"
 
 namespace kda {
 namespace dec {
