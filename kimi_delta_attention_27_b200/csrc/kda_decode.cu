@@ -10,10 +10,10 @@
 //   o  = scale S^T q = scale (S'^T q + beta (k . q) e)
 //
 // The step is bound by HBM: every (request, head) reads its 128 x 128 state and writes it back,
-// against 1.3 KB of token vectors. One CTA per (request, head), 256 threads: warp w owns key rows
-// 16w .. 16w + 15, lane l owns value columns 4l .. 4l + 3, so a warp reads and writes whole
-// 512-byte state rows (fp32; 256 bytes for bf16) with 16-byte accesses, and each thread issues
-// all 16 of its state loads before it uses any of them. S'^T k and S'^T q are reduced over the
+// against 1.3 KB of token vectors. One CTA per (request, head), 256 threads for fp32 states: warp
+// w owns key rows 16w .. 16w + 15, lane l owns value columns 4l .. 4l + 3, so a warp reads and
+// writes whole 512-byte state rows with 16-byte accesses, and each thread issues all 16 of its
+// state loads before it uses any of them. bf16 states: 128 threads, 32 rows per warp (below). S'^T k and S'^T q are reduced over the
 // eight warps in shared memory in one pass; the state is then updated in registers and written
 // back. Each state element is read and written by the same thread, so the output state may be
 // the input state (in place).
@@ -27,9 +27,12 @@ namespace kda {
 namespace dec {
 
 constexpr int D = kHeadDim;
-constexpr int NT = 256;
-constexpr int ROWS = D / (NT / 32);   // key rows per warp
 constexpr float kLog2e = 1.4426950408889634f;
+// threads per CTA: 256 with fp32 states; 128 with bf16 states, which a thread keeps as the loaded
+// bf16 pairs (32 rows x 4 columns in 64 registers) and widens where they are used. A bf16 state
+// is half the bytes for the same fixed work per CTA, so more CTAs have to be resident per SM.
+template <bool kFp32State>
+constexpr int threads() { return kFp32State ? 256 : 128; }
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -45,10 +48,11 @@ __device__ __forceinline__ float ex2(float y) {
 }
 
 template <bool kFp32State>
-__global__ void __launch_bounds__(NT) kda_decode_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(threads<kFp32State>(), kFp32State ? 2 : 3) kda_decode_kernel(DecodeParams p) {
+    constexpr int NT = threads<kFp32State>(), NW = NT / 32, ROWS = D / NW;   // key rows per warp
     __shared__ float ks[D], qs[D], as[D];       // k, q, alpha of this (request, head)
-    __shared__ float4 red[NT / 32][2][D / 4];   // per-warp partial S'^T k and S'^T q
-    __shared__ float kq_part[NT / 32];
+    __shared__ float4 red[NW][2][D / 4];        // per-warp partial S'^T k and S'^T q
+    __shared__ float kq_part[NW];
     __shared__ float4 es[D / 4];                // the retrieval error e, from warp 0
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t bh = blockIdx.x;                               // request * num_heads + head
@@ -57,7 +61,8 @@ __global__ void __launch_bounds__(NT) kda_decode_kernel(DecodeParams p) {
     const int r0 = warp * ROWS, c0 = lane * 4;
 
     // state rows of this thread, loaded before anything else so that they are in flight together
-    float s[ROWS][4];
+    float s[kFp32State ? ROWS : 1][4];
+    uint2 raw[kFp32State ? 1 : ROWS];   // bf16 states: the loaded pairs
     if (p.state_in) {
         if constexpr (kFp32State) {
             const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(p.state_in) + st);
@@ -72,18 +77,29 @@ __global__ void __launch_bounds__(NT) kda_decode_kernel(DecodeParams p) {
         } else {
             const uint2 *src = reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(p.state_in) + st);
 #pragma unroll
-            for (int r = 0; r < ROWS; ++r) {
-                const uint2 x = src[((r0 + r) * D + c0) >> 2];
-                s[r][0] = bf_lo(x.x);
-                s[r][1] = bf_hi(x.x);
-                s[r][2] = bf_lo(x.y);
-                s[r][3] = bf_hi(x.y);
-            }
+            for (int r = 0; r < ROWS; ++r) raw[r] = src[((r0 + r) * D + c0) >> 2];
         }
     } else {
+        if constexpr (kFp32State) {
 #pragma unroll
-        for (int r = 0; r < ROWS; ++r) s[r][0] = s[r][1] = s[r][2] = s[r][3] = 0.f;
+            for (int r = 0; r < ROWS; ++r) s[r][0] = s[r][1] = s[r][2] = s[r][3] = 0.f;
+        } else {
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) raw[r] = make_uint2(0u, 0u);
+        }
     }
+    // row r of S' = Diag(alpha) S, in fp32
+    auto decayed = [&](int r, float a, float (&x)[4]) {
+        if constexpr (kFp32State) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) x[c] = s[r][c] * a;
+        } else {
+            x[0] = bf_lo(raw[r].x) * a;
+            x[1] = bf_hi(raw[r].x) * a;
+            x[2] = bf_lo(raw[r].y) * a;
+            x[3] = bf_hi(raw[r].y) * a;
+        }
+    };
     if (tid < D) {
         ks[tid] = __uint_as_float(static_cast<uint32_t>(p.k[vec + tid]) << 16);
         qs[tid] = __uint_as_float(static_cast<uint32_t>(p.q[vec + tid]) << 16);
@@ -98,12 +114,13 @@ __global__ void __launch_bounds__(NT) kda_decode_kernel(DecodeParams p) {
     float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f}, kq = 0.f;
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
-        const float a = as[r0 + r], kr = ks[r0 + r], qr = qs[r0 + r];
+        const float kr = ks[r0 + r], qr = qs[r0 + r];
+        float x[4];
+        decayed(r, as[r0 + r], x);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            s[r][c] *= a;
-            pk[c] = fmaf(s[r][c], kr, pk[c]);
-            pq[c] = fmaf(s[r][c], qr, pq[c]);
+            pk[c] = fmaf(x[c], kr, pk[c]);
+            pq[c] = fmaf(x[c], qr, pq[c]);
         }
         kq = fmaf(kr, qr, kq);
     }
@@ -115,7 +132,7 @@ __global__ void __launch_bounds__(NT) kda_decode_kernel(DecodeParams p) {
     float rk[4] = {0.f, 0.f, 0.f, 0.f}, rq[4] = {0.f, 0.f, 0.f, 0.f};
     kq = 0.f;
 #pragma unroll
-    for (int w = 0; w < NT / 32; ++w) {
+    for (int w = 0; w < NW; ++w) {
         const float4 a = red[w][0][lane], b = red[w][1][lane];
         rk[0] += a.x;
         rk[1] += a.y;
@@ -154,18 +171,17 @@ __global__ void __launch_bounds__(NT) kda_decode_kernel(DecodeParams p) {
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
         const float bk = beta * ks[r0 + r];
+        float x[4];
+        decayed(r, as[r0 + r], x);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) s[r][c] = fmaf(bk, e[c], s[r][c]);
-    }
-    if constexpr (kFp32State) {
-        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.state_out) + st);
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r) dst[((r0 + r) * D + c0) >> 2] = make_float4(s[r][0], s[r][1], s[r][2], s[r][3]);
-    } else {
-        uint2 *dst = reinterpret_cast<uint2 *>(static_cast<uint16_t *>(p.state_out) + st);
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r)
-            dst[((r0 + r) * D + c0) >> 2] = make_uint2(bf_pack(s[r][0], s[r][1]), bf_pack(s[r][2], s[r][3]));
+        for (int c = 0; c < 4; ++c) x[c] = fmaf(bk, e[c], x[c]);
+        if constexpr (kFp32State) {
+            reinterpret_cast<float4 *>(static_cast<float *>(p.state_out) + st)[((r0 + r) * D + c0) >> 2] =
+                make_float4(x[0], x[1], x[2], x[3]);
+        } else {
+            reinterpret_cast<uint2 *>(static_cast<uint16_t *>(p.state_out) + st)[((r0 + r) * D + c0) >> 2] =
+                make_uint2(bf_pack(x[0], x[1]), bf_pack(x[2], x[3]));
+        }
     }
 }
 
@@ -174,11 +190,11 @@ __global__ void __launch_bounds__(NT) kda_decode_kernel(DecodeParams p) {
 cudaError_t launch_decode(const DecodeParams &p, int64_t units, cudaStream_t stream) {
     if (units <= 0) return cudaSuccess;
     if (units > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    const dim3 grid(static_cast<unsigned>(units)), block(dec::NT);
+    const dim3 grid(static_cast<unsigned>(units));
     if (p.state_fp32)
-        dec::kda_decode_kernel<true><<<grid, block, 0, stream>>>(p);
+        dec::kda_decode_kernel<true><<<grid, dec::threads<true>(), 0, stream>>>(p);
     else
-        dec::kda_decode_kernel<false><<<grid, block, 0, stream>>>(p);
+        dec::kda_decode_kernel<false><<<grid, dec::threads<false>(), 0, stream>>>(p);
     return cudaGetLastError();
 }
 
