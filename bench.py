@@ -44,6 +44,13 @@ def pages_flops(tokens: int, H: int) -> float:
     return float(tokens) * H * FLOPS_PER_TOKEN_HEAD
 
 
+def decode_unit_bytes(state_dtype: str) -> int:
+    """Algorithmic HBM bytes of one decode step for one (request, head): the 128 x 128 state
+    read and written, q, k, v and out (bf16), g (fp32) and beta."""
+    esz = 4 if state_dtype == "fp32" else 2
+    return 2 * D * D * esz + 4 * D * 2 + D * 4 + 4
+
+
 def state_bytes(N, H, init_dt, final_dt) -> int:
     b = 0
     for dt in (init_dt, final_dt):
@@ -441,9 +448,7 @@ def decode_main(args):
     clocks = sampler.stop()
     ms_per_step = t0.elapsed_time(t1) / steps
     launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    esz = 4 if sdt == "fp32" else 2
-    # per (request, head): the state read and written, q, k, v, out (bf16), g (fp32), beta
-    unit_bytes = 2 * D * D * esz + 4 * D * 2 + D * 4 + 4
+    unit_bytes = decode_unit_bytes(sdt)
     alg_bytes = B * H * unit_bytes
     peaks = load_peaks()
     achieved = alg_bytes / (launch_ms / 1e3) / 1e9
