@@ -1,4 +1,4 @@
-"""fp64 CPU oracle for the Kimi Delta Attention forward pass.
+"""fp64 CPU oracle for the Kimi Delta Attention forward pass (and its gradients).
 
 TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke()``
 and by the CPU-baseline leg of ``bench.py``. The product package never imports
@@ -58,6 +58,10 @@ def _declare(lib):
     lib.kda_oracle_fwd.argtypes = [P, P, P, P, P, ctypes.c_double, P, ctypes.c_int64,
                                    ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                    P, P, P, ctypes.c_int]
+    i64 = ctypes.c_int64
+    lib.kda_oracle_bwd.restype = ctypes.c_int
+    lib.kda_oracle_bwd.argtypes = [P, P, P, P, P, ctypes.c_double, P, i64, i64, i64, i64,
+                                   P, P, P, P, P, P, P, P, P, ctypes.c_int]
 
 
 def _f32(x) -> np.ndarray:
@@ -124,3 +128,46 @@ def kda_oracle(q, k, v, g, beta, scale, cu_seqlens=None, h0=None, nthreads=None,
     if rc != 0:
         raise ValueError("kda_oracle_fwd rejected its arguments")
     return out.reshape(*lead, Dv), hT
+
+
+def _cu_of(qa, cu_seqlens):
+    if cu_seqlens is None:
+        B, T = (qa.shape[0], qa.shape[1]) if qa.ndim == 4 else (1, qa.shape[0])
+        return np.arange(B + 1, dtype=np.int64) * T
+    return np.ascontiguousarray(np.asarray(
+        cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int64))
+
+
+def kda_oracle_bwd(q, k, v, g, beta, scale, dout, cu_seqlens=None, h0=None, dhT=None, nthreads=None,
+                   lib_path: str | None = None):
+    """Gradients of ``sum(dout * out) + sum(dhT * hT)`` of the fp64 recurrence.
+
+    Same inputs and layouts as ``kda_oracle`` (taken as float64 here, exactly), plus ``dout``
+    shaped like ``out`` and ``dhT`` shaped like ``hT`` (or None). Returns a dict of float64
+    arrays: dq, dk, dv, dg, dbeta shaped like their inputs, and dh0 [N, H, Dk, Dv].
+    """
+    qa, ka, va, ga, ba, da = (_f64(t) for t in (q, k, v, g, beta, dout))
+    cu = _cu_of(qa, cu_seqlens)
+    Dk, Dv, H = qa.shape[-1], va.shape[-1], qa.shape[-2]
+    N = len(cu) - 1
+    shapes = dict(dq=qa.shape, dk=ka.shape, dv=va.shape, dg=ga.shape, dbeta=ba.shape)
+    qa, ka, ga = (a.reshape(-1, H, Dk) for a in (qa, ka, ga))
+    va, da = va.reshape(-1, H, Dv), da.reshape(-1, H, Dv)
+    ba = ba.reshape(-1, H)
+    if cu[-1] > qa.shape[0]:
+        raise ValueError("cu_seqlens runs past the packed tensors")
+    h0a = None if h0 is None else _f64(h0).reshape(N, H, Dk, Dv)
+    dhTa = None if dhT is None else _f64(dhT).reshape(N, H, Dk, Dv)
+    out = {n: np.zeros(qa.shape if n in ("dq", "dk", "dg") else (va.shape if n == "dv" else ba.shape))
+           for n in ("dq", "dk", "dv", "dg", "dbeta")}
+    dh0 = np.zeros((N, H, Dk, Dv))
+    lib = _load(lib_path)
+    P = lambda a: None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+    rc = lib.kda_oracle_bwd(P(qa), P(ka), P(va), P(ga), P(ba), float(scale), P(cu), N, H, Dk, Dv,
+                            P(h0a), P(da), P(dhTa), P(out["dq"]), P(out["dk"]), P(out["dv"]),
+                            P(out["dg"]), P(out["dbeta"]), P(dh0), int(nthreads or os.cpu_count() or 1))
+    if rc != 0:
+        raise ValueError("kda_oracle_bwd rejected its arguments")
+    res = {n: a.reshape(shapes[n]) for n, a in out.items()}
+    res["dh0"] = dh0
+    return res
