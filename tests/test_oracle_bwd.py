@@ -8,7 +8,9 @@ page, chapter 4: S_t = (Diag(alpha_t) - beta_t k_t (k_t (.) alpha_t)^T) S_{t-1}
 against the pinned C forward oracle. Central finite differences, element by
 element on tiny cases and along random directions on a case that crosses the
 backward's 64-token checkpoints, must match the analytic gradients; so must
-a handful of exact special cases.
+a handful of exact special cases. A chunkwise backward of the chunk form the
+kernels use (the algebra a backward kernel would follow) must agree with it for
+chunk sizes 1 to 64 and ragged sequences.
 """
 import numpy as np
 import pytest
@@ -138,3 +140,99 @@ def test_gradients_are_linear_in_the_cotangents():
     g12 = grads(c, dout=c["dout"] + d2o, dhT=c["dhT"] + d2s)
     for n in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
         assert np.allclose(g12[n], g1[n] + g2[n], rtol=1e-12, atol=1e-12), n
+
+
+def chunkwise_backward(c, C):
+    """fp64 chunkwise backward of the chunk form the kernels use (per chunk, Gam the in-chunk
+    running log-decay, Kd = K e^Gam, Qd = Q e^Gam, Kn = K e^-Gam, Kt = K e^(Gam_last - Gam)):
+
+        A_kk = strict_lower(Diag(beta) Kd Kn^T),  A_qk = lower(Qd Kn^T),  T = (I + A_kk)^-1
+        X = V - Kd S0,  D = T Diag(beta) X,  O = scale (Qd S0 + A_qk D)
+        S1 = Diag(e^Gam_last) S0 + Kt^T D
+
+    written backwards chunk by chunk from dO and the final-state gradient. The blueprint of a
+    chunkwise backward kernel; here it pins, and is pinned by, the token-by-token backward."""
+    q, k, v, g, beta, cu, scale = c["q"], c["k"], c["v"], c["g"], c["beta"], c["cu"], c["scale"]
+    Ttot, H, Dk = q.shape
+    Dv = v.shape[-1]
+    N = len(cu) - 1
+    res = {n: np.zeros_like(c[n]) for n in ("q", "k", "v", "g", "beta")}
+    dh0 = np.zeros((N, H, Dk, Dv))
+    for s in range(N):
+        for h in range(H):
+            bounds = [(t0, min(t0 + C, cu[s + 1])) for t0 in range(cu[s], cu[s + 1], C)]
+            # forward: the state at every chunk start
+            S = np.zeros((Dk, Dv)) if c["h0"] is None else c["h0"][s, h].copy()
+            starts, parts = [], []
+            for t0, t1 in bounds:
+                K, Q, V = k[t0:t1, h], q[t0:t1, h], v[t0:t1, h]
+                Gam = np.cumsum(g[t0:t1, h], axis=0)
+                b = beta[t0:t1, h]
+                Kd, Qd, Kn = K * np.exp(Gam), Q * np.exp(Gam), K * np.exp(-Gam)
+                Kt = K * np.exp(Gam[-1] - Gam)
+                B = Kd @ Kn.T
+                Akk = np.tril(b[:, None] * B, -1)
+                Aqk = np.tril(Qd @ Kn.T, 0)
+                T = np.linalg.inv(np.eye(len(b)) + Akk)
+                X = V - Kd @ S
+                Dl = T @ (b[:, None] * X)
+                starts.append(S.copy())
+                parts.append((K, Q, Gam, b, Kd, Qd, Kn, Kt, B, Aqk, T, X, Dl))
+                S = np.exp(Gam[-1])[:, None] * S + Kt.T @ Dl
+            # backward, last chunk first
+            dS = c["dhT"][s, h].copy()
+            for (t0, t1), S0, (K, Q, Gam, b, Kd, Qd, Kn, Kt, B, Aqk, T, X, Dl) in \
+                    reversed(list(zip(bounds, starts, parts))):
+                dO = c["dout"][t0:t1, h]
+                eC = np.exp(Gam[-1])
+                # O = scale (Qd S0 + Aqk D)
+                dQd = scale * dO @ S0.T
+                dS0 = scale * Qd.T @ dO
+                dAqk = np.tril(scale * dO @ Dl.T, 0)
+                dD = scale * Aqk.T @ dO
+                # S1 = Diag(e^Gam_last) S0 + Kt^T D
+                dS0 += eC[:, None] * dS
+                dGlast = eC * (dS * S0).sum(axis=1)
+                dKt = Dl @ dS.T
+                dD += Kt @ dS
+                # D = T Diag(beta) X
+                Tp = T * b[None, :]
+                dTp = dD @ X.T
+                dX = Tp.T @ dD
+                dV = dX
+                dKd = -dX @ S0.T
+                dS0 -= Kd.T @ dX
+                db = (dTp * T).sum(axis=0)
+                dT = dTp * b[None, :]
+                # T = (I + Akk)^-1 ; Akk = strict_lower(Diag(beta) B)
+                dAkk = np.tril(-T.T @ dT @ T.T, -1)
+                db += (dAkk * B).sum(axis=1)
+                dB = b[:, None] * dAkk
+                dKd += dB @ Kn
+                dKn = dB.T @ Kd
+                # Aqk = lower(Qd Kn^T)
+                dQd += dAqk @ Kn
+                dKn += dAqk.T @ Qd
+                # the decayed factors back to K, Q and the running log-decay
+                dK = dKd * np.exp(Gam) + dKn * np.exp(-Gam) + dKt * np.exp(Gam[-1] - Gam)
+                dQ = dQd * np.exp(Gam)
+                dGam = dKd * Kd + dQd * Qd - dKn * Kn - dKt * Kt
+                dGam[-1] += dGlast + (dKt * Kt).sum(axis=0)
+                res["k"][t0:t1, h] = dK
+                res["q"][t0:t1, h] = dQ
+                res["v"][t0:t1, h] = dV
+                res["beta"][t0:t1, h] = db
+                res["g"][t0:t1, h] = np.cumsum(dGam[::-1], axis=0)[::-1]   # Gam = cumsum(g)
+                dS = dS0
+            dh0[s, h] = dS
+    return {"d" + n: a for n, a in res.items()} | {"dh0": dh0}
+
+
+@pytest.mark.parametrize("C", [1, 4, 16, 64])
+def test_chunkwise_backward_equals_the_token_by_token_backward(C):
+    c = case(11, [70, 5, 0, 33], H=2, Dk=6, Dv=5)
+    ref = grads(c)
+    got = chunkwise_backward(c, C)
+    for n in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
+        err = np.abs(got[n] - ref[n]).max() / max(1.0, np.abs(ref[n]).max())
+        assert err <= 1e-10, f"C={C} {n}: {err:.2e}"
