@@ -321,3 +321,31 @@ def test_mutants_are_caught(mutant, tmp_path, oracle_mod):
         except AssertionError:
             failed.append(check.__name__)
     assert failed, f"planted mistake {mutant} passed every pin"
+
+
+def test_segments_compose_through_their_affine_maps():
+    """The state-update equation is affine in the state, so a segment maps S_in to M S_in + B,
+    with M the final state of a run from the identity with v = 0 and B the final state of a run
+    from zero. Scanning (M, B) over segments and re-running each from the scanned state must
+    reproduce one run over the whole sequence (the construction of a segment-parallel scan)."""
+    rng = np.random.default_rng(21)
+    T, H, D = 300, 2, 16
+    f = lambda *s: rng.normal(size=s).astype(np.float32)
+    q, v = f(1, T, H, D), f(1, T, H, D)
+    k = (f(1, T, H, D) / 4).astype(np.float32)
+    g = (-np.abs(f(1, T, H, D)) * 0.1).astype(np.float32)
+    beta = rng.uniform(0, 1, size=(1, T, H)).astype(np.float32)
+    h0 = rng.normal(size=(1, H, D, D)) * 0.3
+    ref_out, ref_hT = oracle.kda_oracle(q, k, v, g, beta, 0.5, h0=h0)
+    eye = np.broadcast_to(np.eye(D), (1, H, D, D)).copy()
+    S, outs = h0.copy(), []
+    for a, b in ((0, 100), (100, 230), (230, 300)):
+        sl = lambda x: np.ascontiguousarray(x[:, a:b])
+        _, M = oracle.kda_oracle(sl(q), sl(k), np.zeros_like(sl(v)), sl(g), sl(beta), 0.5, h0=eye)
+        _, B = oracle.kda_oracle(sl(q), sl(k), sl(v), sl(g), sl(beta), 0.5)
+        o, _ = oracle.kda_oracle(sl(q), sl(k), sl(v), sl(g), sl(beta), 0.5, h0=S)
+        outs.append(o)
+        S = np.einsum("hij,hjk->hik", M[0], S[0])[None] + B
+    out = np.concatenate(outs, axis=1)
+    assert np.abs(out - ref_out).max() <= 1e-12 * np.abs(ref_out).max()
+    assert np.abs(S - ref_hT).max() <= 1e-12 * np.abs(ref_hT).max()
