@@ -33,6 +33,7 @@
 #ifndef KDA_H_
 #define KDA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -53,7 +54,11 @@ typedef enum {
     KDA_ERR_TOO_LARGE = 8,         /* sizes exceed what the library indexes              */
     KDA_ERR_TIMEOUT = 9,           /* a kernel gave up on a bounded wait (see kda_device_error) */
     KDA_ERR_NOALLOC_LIMIT = 10,    /* kda_fwd_noalloc: more (sequence, head) pairs than its scratch holds */
-    KDA_ERR_STATE_OVERLAP = 11     /* kda_decode: distinct state_in and state_out buffers overlap */
+    KDA_ERR_STATE_OVERLAP = 11,    /* kda_decode: distinct state_in and state_out buffers overlap */
+    KDA_ERR_BAD_CU_SEQLENS = 12,   /* (kda_device_error) cu_seqlens was not 0, ..., seq_len non-decreasing */
+    KDA_ERR_INTERNAL = 13,         /* (kda_device_error) a kernel ran where its scratch has no slot for it */
+    KDA_ERR_BAD_OPTION = 14,       /* kda_fwd_ex: unknown gate kind or flag bit */
+    KDA_ERR_WORKSPACE = 15         /* kda_fwd_segmented: workspace smaller than it needs */
 } kda_status;
 
 typedef enum { KDA_DTYPE_NONE = 0, KDA_DTYPE_BF16 = 1, KDA_DTYPE_FP32 = 2 } kda_dtype;
@@ -76,12 +81,15 @@ typedef enum { KDA_DTYPE_NONE = 0, KDA_DTYPE_BF16 = 1, KDA_DTYPE_FP32 = 2 } kda_
  *   cu_seqlens != NULL : batch must be 1; cu_seqlens is a DEVICE int32 array of
  *                        num_seqs + 1 offsets into the seq_len packed tokens,
  *                        cu_seqlens[0] = 0, non-decreasing, last = seq_len;
- *                        num_seqs_eff = num_seqs. Entries are clamped into
- *                        [0, seq_len] and a decreasing pair is read as an empty
- *                        sequence, so a malformed table cannot make the kernel
- *                        access memory out of bounds (its results are then
- *                        unspecified). Zero-length sequences are allowed: their
- *                        final state equals their initial state.
+ *                        num_seqs_eff = num_seqs. The table lives on the
+ *                        device, so it is checked there: a malformed table
+ *                        raises KDA_ERR_BAD_CU_SEQLENS in the device error word
+ *                        (read by kda_device_error). Its entries are clamped
+ *                        into [0, seq_len] and a decreasing pair is read as an
+ *                        empty sequence, so the kernel still accesses no memory
+ *                        out of bounds; the results are then unspecified.
+ *                        Zero-length sequences are allowed: their final state
+ *                        equals their initial state.
  *
  * State:
  *   initial_state == NULL (initial_dtype ignored) means zero initial states.
@@ -93,6 +101,14 @@ typedef enum { KDA_DTYPE_NONE = 0, KDA_DTYPE_BF16 = 1, KDA_DTYPE_FP32 = 2 } kda_
  * scale multiplies the output (o_t = scale * S_t^T q_t); callers normally
  * pass 1/sqrt(128).
  *
+ * Gate range: g may be any value <= 0, including -inf (alpha = 0). The kernel
+ * raises per-token log-decays below -10 to -10 (alpha >= e^-10 = 4.5e-5): a
+ * channel that keeps less than that of its state per token has forgotten it
+ * to below the precision of its bf16 operands either way, and the change in
+ * any output is bounded by e^-10 relative to the state it reads. Chunks whose
+ * decay over either half exceeds 2^-100 on some channel take a slower path
+ * with one decay anchor per 16 tokens instead of one per chunk.
+ *
  * head_dim_k and head_dim_v must both be 128. All tensor pointers must be
  * 16-byte aligned (cu_seqlens 4-byte). Returns KDA_OK once the work is
  * enqueued.
@@ -103,6 +119,80 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
                    int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
                    kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype,
                    void *out, kda_stream_t stream);
+
+/*
+ * kda_fwd_ex -- kda_fwd with the input variants of the same operator.
+ *
+ * The Kimi Linear feature page (chapter 4, "innovation 1") defines the forget
+ * gate per channel and sets it against Gated DeltaNet's single decay per token
+ * (the Kimi Delta Attention review page, "Kimi Delta Attention" section, makes
+ * the same contrast). The workloads give q and k L2-normalised and g as a
+ * log-sigmoid; these variants take those steps, or cheaper inputs, into the
+ * kernel instead of a separate pass over HBM:
+ *
+ *   gate_kind  KDA_GATE_FP32        g fp32 [batch, seq_len, num_heads, 128] (kda_fwd)
+ *              KDA_GATE_BF16        g bf16 [batch, seq_len, num_heads, 128]: 256 fewer
+ *                                   bytes to read per token and head (1284 instead of 1540)
+ *              KDA_GATE_SCALAR_FP32 g fp32 [batch, seq_len, num_heads]: one decay per token
+ *                                   and head, the same on every channel (Gated DeltaNet);
+ *                                   4-byte alignment suffices
+ *   flags      KDA_FLAG_L2NORM_QK        q and k are divided by their L2 norm over the 128
+ *                                        channels of each token and head (a zero vector
+ *                                        stays zero) before use
+ *              KDA_FLAG_GATE_LOGSIGMOID  g holds the gate's pre-activation x, and
+ *                                        log alpha = logsigmoid(x) = -log(1 + e^-x)
+ *
+ * Everything else, and every status, is as for kda_fwd; an unknown gate_kind or
+ * flag bit returns KDA_ERR_BAD_OPTION.
+ */
+#define KDA_GATE_FP32 0
+#define KDA_GATE_BF16 1
+#define KDA_GATE_SCALAR_FP32 2
+#define KDA_FLAG_L2NORM_QK 1u
+#define KDA_FLAG_GATE_LOGSIGMOID 2u
+kda_status kda_fwd_ex(const void *q, const void *k, const void *v, const void *g, int32_t gate_kind,
+                      const float *beta, float scale, const int32_t *cu_seqlens, int32_t num_seqs,
+                      int32_t batch, int64_t seq_len, int32_t num_heads, int32_t head_dim_k,
+                      int32_t head_dim_v, const void *initial_state, kda_dtype initial_dtype,
+                      void *final_state, kda_dtype final_dtype, void *out, uint32_t flags,
+                      kda_stream_t stream);
+
+/*
+ * kda_fwd_segmented -- kda_fwd over long sequences split into pieces that run at
+ * once, for batches with few (sequence, head) pairs.
+ *
+ * The Kimi Linear feature page (chapter 8) keeps the state at a fixed 128 x 128
+ * per head however long the context (1M tokens on the release page). kda_fwd runs
+ * each (sequence, head) pair's chunks in order on one set of SMs, so a batch of few
+ * pairs leaves most of the GPU idle. The recurrence is affine in the state: a piece
+ * of a sequence maps its entering state S to M S + B. This entry point splits every
+ * row into pieces of segment_len tokens and makes three launches on `stream`:
+ *   1. every piece twice, with no output: from a zero state (giving B) and from the
+ *      identity with v = 0 (giving M); all pieces of all rows at once;
+ *   2. the scan S_0 = initial state, S_(j+1) = M_j S_j + B_j, per row and head;
+ *   3. every piece again from its S_j, writing the outputs and, for the last piece,
+ *      the row's final state.
+ * That is about three times kda_fwd's work, done in parallel over the pieces: it
+ * pays when batch * num_heads is small next to the number of SMs.
+ *
+ * Arguments and layouts are kda_fwd's for fixed-length rows (no cu_seqlens), plus:
+ *   segment_len     tokens per piece, a positive multiple of 64; a row that fits in
+ *                   one piece runs as in kda_fwd;
+ *   workspace       caller-owned device memory, 256-byte aligned, of at least
+ *                   kda_fwd_segmented_workspace(batch, seq_len, num_heads,
+ *                   segment_len) bytes (three fp32 states per piece and head); its
+ *                   contents on entry do not matter. KDA_ERR_WORKSPACE if smaller.
+ * Results agree with kda_fwd's to the rounding of the bf16 state copies the
+ * products use; the pieces' states are carried in fp32. A bad segment_len returns
+ * KDA_ERR_BAD_SHAPE, and kda_fwd_segmented_workspace returns 0 for one.
+ */
+size_t kda_fwd_segmented_workspace(int32_t batch, int64_t seq_len, int32_t num_heads, int64_t segment_len);
+kda_status kda_fwd_segmented(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, float scale, int32_t batch, int64_t seq_len,
+                             int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v,
+                             const void *initial_state, kda_dtype initial_dtype, void *final_state,
+                             kda_dtype final_dtype, void *out, int64_t segment_len, void *workspace,
+                             size_t workspace_bytes, kda_stream_t stream);
 
 /*
  * kda_fwd_noalloc -- kda_fwd for callers that cannot allocate device memory.
@@ -176,11 +266,15 @@ kda_status kda_decode(const void *q, const void *k, const void *v, const float *
 
 /*
  * kda_device_error -- synchronise the current device, then read and clear the
- * library's device-side error word. Every wait inside the kernels is bounded
- * (a few seconds); a kernel that gives up raises this word and returns early
- * instead of hanging, leaving its outputs unspecified. Returns KDA_ERR_TIMEOUT
- * if that happened on this device since the previous call, KDA_OK otherwise,
- * KDA_ERR_CUDA if the device could not be synchronised or read.
+ * library's device-side error word, which the kernels raise instead of
+ * faulting or hanging. Since the previous call on this device, if any kernel:
+ *  - found cu_seqlens malformed (see kda_fwd): KDA_ERR_BAD_CU_SEQLENS;
+ *  - gave up on a bounded wait (every wait is bounded, a few seconds) and
+ *    returned early, leaving its outputs unspecified: KDA_ERR_TIMEOUT;
+ *  - ran a chain CTA on an SM id beyond the scratch pool's rings (none exists
+ *    on a B200) and returned at once: KDA_ERR_INTERNAL;
+ * the first of these in this order is returned, else KDA_OK; KDA_ERR_CUDA if
+ * the device could not be synchronised or read.
  */
 kda_status kda_device_error(void);
 

@@ -25,12 +25,15 @@ bool device_is_sm100(int *err) {
 
 // Validate the arguments of kda_fwd / kda_fwd_noalloc and fill the kernel parameters.
 // Returns KDA_OK with p->num_seqs == 0 when there is nothing to do.
-kda_status prepare(const void *q, const void *k, const void *v, const float *g, const float *beta, float scale,
+kda_status prepare(const void *q, const void *k, const void *v, const void *g, const float *beta, float scale,
                    const int32_t *cu_seqlens, int32_t num_seqs, int32_t batch, int64_t seq_len,
                    int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v, const void *initial_state,
                    kda_dtype initial_dtype, void *final_state, kda_dtype final_dtype, void *out,
-                   bool noalloc, kda::FwdParams *p, int64_t *rows_out) {
+                   bool noalloc, int32_t gate_kind, uint32_t flags, kda::FwdParams *p, int64_t *rows_out) {
     p->num_seqs = 0;
+    if (gate_kind != KDA_GATE_FP32 && gate_kind != KDA_GATE_BF16 && gate_kind != KDA_GATE_SCALAR_FP32)
+        return KDA_ERR_BAD_OPTION;
+    if (flags & ~static_cast<uint32_t>(KDA_FLAG_L2NORM_QK | KDA_FLAG_GATE_LOGSIGMOID)) return KDA_ERR_BAD_OPTION;
     if (head_dim_k != kda::kHeadDim || head_dim_v != kda::kHeadDim) return KDA_ERR_BAD_SHAPE;
     if (batch < 0 || seq_len < 0 || num_heads < 1 || num_seqs < 0) return KDA_ERR_BAD_SHAPE;
     if (cu_seqlens && batch != 1) return KDA_ERR_VARLEN_BATCH;
@@ -43,7 +46,8 @@ kda_status prepare(const void *q, const void *k, const void *v, const float *g, 
     const int64_t rows = cu_seqlens ? seq_len : static_cast<int64_t>(batch) * seq_len;
     if (rows > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_NULL_PTR;
     if (cu_seqlens && !(reinterpret_cast<uintptr_t>(cu_seqlens) % 4 == 0)) return KDA_ERR_BAD_ALIGNMENT;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(out) ||
+    const bool g_ok = gate_kind == KDA_GATE_SCALAR_FP32 ? (reinterpret_cast<uintptr_t>(g) & 3u) == 0 : aligned16(g);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !g_ok || !aligned16(out) ||
         !aligned16(initial_state) || !aligned16(final_state) ||
         (reinterpret_cast<uintptr_t>(beta) & 3u))
         return KDA_ERR_BAD_ALIGNMENT;
@@ -71,6 +75,12 @@ kda_status prepare(const void *q, const void *k, const void *v, const float *g, 
     p->hT = final_state;
     p->hT_fp32 = final_dtype == KDA_DTYPE_FP32;
     p->out = static_cast<uint16_t *>(out);
+    p->gate_mode = gate_kind;
+    p->flags = flags;
+    p->seg_len = 0;
+    p->seg_count = 0;
+    p->mode = kda::kModePlain;
+    p->hT_aux = nullptr;
     *rows_out = rows;
     return KDA_OK;
 }
@@ -95,11 +105,19 @@ const char *kda_status_string(kda_status s) {
             return "KDA_ERR_NOALLOC_LIMIT: kda_fwd_noalloc takes at most 32 (sequence, head) pairs per call";
         case KDA_ERR_STATE_OVERLAP:
             return "KDA_ERR_STATE_OVERLAP: kda_decode state_in and state_out overlap without being the same buffer";
+        case KDA_ERR_BAD_CU_SEQLENS:
+            return "KDA_ERR_BAD_CU_SEQLENS: cu_seqlens must run 0, ..., seq_len without decreasing";
+        case KDA_ERR_INTERNAL:
+            return "KDA_ERR_INTERNAL: a kernel ran on an SM beyond its scratch pool and stopped";
+        case KDA_ERR_BAD_OPTION:
+            return "KDA_ERR_BAD_OPTION: unknown gate kind or flag";
+        case KDA_ERR_WORKSPACE:
+            return "KDA_ERR_WORKSPACE: the workspace is smaller than kda_fwd_segmented_workspace() asks";
     }
     return "KDA_ERR_UNKNOWN";
 }
 
-int32_t kda_version(void) { return (1 << 16) | 2; }
+int32_t kda_version(void) { return (1 << 16) | 3; }
 
 kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
                    const float *beta, float scale, const int32_t *cu_seqlens,
@@ -111,9 +129,89 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
     int64_t rows = 0;
     const kda_status st = prepare(q, k, v, g, beta, scale, cu_seqlens, num_seqs, batch, seq_len, num_heads,
                                   head_dim_k, head_dim_v, initial_state, initial_dtype, final_state,
-                                  final_dtype, out, false, &p, &rows);
+                                  final_dtype, out, false, KDA_GATE_FP32, 0u, &p, &rows);
     if (st != KDA_OK || p.num_seqs == 0) return st;
     const cudaError_t err = kda::launch_fwd_tc(p, rows, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_fwd_ex(const void *q, const void *k, const void *v, const void *g, int32_t gate_kind,
+                      const float *beta, float scale, const int32_t *cu_seqlens, int32_t num_seqs,
+                      int32_t batch, int64_t seq_len, int32_t num_heads, int32_t head_dim_k,
+                      int32_t head_dim_v, const void *initial_state, kda_dtype initial_dtype,
+                      void *final_state, kda_dtype final_dtype, void *out, uint32_t flags,
+                      kda_stream_t stream) {
+    kda::FwdParams p;
+    int64_t rows = 0;
+    const kda_status st = prepare(q, k, v, g, beta, scale, cu_seqlens, num_seqs, batch, seq_len, num_heads,
+                                  head_dim_k, head_dim_v, initial_state, initial_dtype, final_state,
+                                  final_dtype, out, false, gate_kind, flags, &p, &rows);
+    if (st != KDA_OK || p.num_seqs == 0) return st;
+    const cudaError_t err = kda::launch_fwd_tc(p, rows, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+size_t kda_fwd_segmented_workspace(int32_t batch, int64_t seq_len, int32_t num_heads, int64_t segment_len) {
+    if (batch < 0 || seq_len < 0 || num_heads < 1 || segment_len < kda::kChunk || segment_len % kda::kChunk)
+        return 0;
+    const int64_t pieces = (seq_len + segment_len - 1) / segment_len;
+    return static_cast<size_t>(3) * static_cast<size_t>(batch) * static_cast<size_t>(pieces) *
+           static_cast<size_t>(num_heads) * kda::kHeadDim * kda::kHeadDim * sizeof(float);
+}
+
+kda_status kda_fwd_segmented(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, float scale, int32_t batch, int64_t seq_len,
+                             int32_t num_heads, int32_t head_dim_k, int32_t head_dim_v,
+                             const void *initial_state, kda_dtype initial_dtype, void *final_state,
+                             kda_dtype final_dtype, void *out, int64_t segment_len, void *workspace,
+                             size_t workspace_bytes, kda_stream_t stream) {
+    if (segment_len < kda::kChunk || segment_len % kda::kChunk) return KDA_ERR_BAD_SHAPE;
+    kda::FwdParams p;
+    int64_t rows = 0;
+    kda_status st = prepare(q, k, v, g, beta, scale, nullptr, 0, batch, seq_len, num_heads, head_dim_k,
+                            head_dim_v, initial_state, initial_dtype, final_state, final_dtype, out, false,
+                            KDA_GATE_FP32, 0u, &p, &rows);
+    if (st != KDA_OK || p.num_seqs == 0) return st;
+    const int64_t pieces = (seq_len + segment_len - 1) / segment_len;
+    if (pieces <= 1) {
+        const cudaError_t err = kda::launch_fwd_tc(p, rows, reinterpret_cast<cudaStream_t>(stream));
+        return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
+    const int64_t units = static_cast<int64_t>(batch) * pieces;
+    if (units * num_heads > (int64_t(1) << 28) || units > 0x7fffffffLL) return KDA_ERR_TOO_LARGE;
+    const size_t need = kda_fwd_segmented_workspace(batch, seq_len, num_heads, segment_len);
+    if (!workspace) return KDA_ERR_NULL_PTR;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KDA_ERR_BAD_ALIGNMENT;
+    if (workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    const size_t per = need / 3 / sizeof(float);
+    float *Mb = static_cast<float *>(workspace), *Bb = Mb + per, *Sin = Bb + per;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // 1. every piece's affine map: B from a zero state, M from the identity with v = 0
+    kda::FwdParams pa = p;
+    pa.num_seqs = static_cast<int32_t>(units);
+    pa.seg_len = segment_len;
+    pa.seg_count = static_cast<int32_t>(pieces);
+    pa.mode = kda::kModeAffine;
+    pa.h0 = nullptr;
+    pa.hT = Bb;
+    pa.hT_fp32 = 1;
+    pa.hT_aux = Mb;
+    cudaError_t err = kda::launch_fwd_tc(pa, rows, s);
+    // 2. the states entering the pieces
+    if (err == cudaSuccess)
+        err = kda::launch_segment_scan(initial_state, initial_dtype == KDA_DTYPE_FP32, Mb, Bb, Sin, batch,
+                                       static_cast<int32_t>(pieces), num_heads, s);
+    // 3. every piece from its entering state: the outputs, and each row's final state
+    if (err == cudaSuccess) {
+        kda::FwdParams pp = pa;
+        pp.mode = kda::kModePlain;
+        pp.h0 = Sin;
+        pp.h0_fp32 = 1;
+        pp.hT = final_state;
+        pp.hT_fp32 = final_dtype == KDA_DTYPE_FP32;
+        pp.hT_aux = nullptr;
+        err = kda::launch_fwd_tc(pp, rows, s);
+    }
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -127,7 +225,7 @@ kda_status kda_fwd_noalloc(const void *q, const void *k, const void *v, const fl
     int64_t rows = 0;
     const kda_status st = prepare(q, k, v, g, beta, scale, cu_seqlens, num_seqs, batch, seq_len, num_heads,
                                   head_dim_k, head_dim_v, initial_state, initial_dtype, final_state,
-                                  final_dtype, out, true, &p, &rows);
+                                  final_dtype, out, true, KDA_GATE_FP32, 0u, &p, &rows);
     if (st != KDA_OK || p.num_seqs == 0) return st;
     const cudaError_t err = kda::launch_fwd_tc_noalloc(p, rows, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -176,7 +274,10 @@ kda_status kda_device_error(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return KDA_ERR_CUDA;
     unsigned int v = 0;
     if (kda::read_and_clear_device_error(&v) != cudaSuccess) return KDA_ERR_CUDA;
-    return v ? KDA_ERR_TIMEOUT : KDA_OK;
+    if (v & kda::kErrCuSeqlens) return KDA_ERR_BAD_CU_SEQLENS;
+    if (v & kda::kErrTimeout) return KDA_ERR_TIMEOUT;
+    if (v & kda::kErrRingIndex) return KDA_ERR_INTERNAL;
+    return KDA_OK;
 }
 
 }  // extern "C"

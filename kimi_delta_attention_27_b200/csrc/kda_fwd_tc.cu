@@ -38,6 +38,7 @@
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -47,6 +48,13 @@
 namespace kda {
 
 __device__ unsigned int g_kda_device_error = 0;
+
+#ifdef KDA_TEST_HOOKS
+// Test-only build (never the product library): the publisher of chunk
+// g_kda_test_skip_chunk leaves that chunk's ring slot unsignalled, so that the
+// chain CTA's bounded wait for it runs out and the kernel winds down early.
+__device__ int g_kda_test_skip_chunk = -1;
+#endif
 
 #ifdef KDA_TRACE
 // Development-only timeline: when built with -DKDA_TRACE, the first cluster
@@ -134,7 +142,10 @@ constexpr uint32_t M_BETA = 256, M_EGA = 512;                  // 64, 128 floats
 constexpr uint32_t M_BETAQ = 1024, M_CHUNKQ = 1536, M_CONSUMED = 1552, M_NEXT = 1568;
 constexpr uint32_t M_DEC = 2048;                               // 2 x 128 floats (e^Gl, part of the set)
 constexpr uint32_t M_TMEM = 3072, M_ABORT = 3088, M_SMID = 3104;
-constexpr uint32_t MISC_BYTES = 3584;
+constexpr uint32_t M_HTINFO = 3136;   // chain: where the final state goes (pointer, offset, flags)
+constexpr uint32_t M_GSCALQ = 3584;                            // prep: 2 x 64 floats, a per-token gate
+constexpr uint32_t M_INVN = 4096;     // prep: 1 / ||q||, 1 / ||k|| of the chunk's 64 rows (128 floats)
+constexpr uint32_t MISC_BYTES = 4608;
 constexpr uint32_t SMEM_USED = (CH_MISC > PR_MISC ? CH_MISC : PR_MISC) + MISC_BYTES;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 
@@ -169,7 +180,16 @@ static_assert(CB_COUNT * 8 <= M_BETA && PB_COUNT * 8 <= M_BETA, "barrier area");
 // chain: C1^T (two buffers), C3^T, S'^T (bf16 pairs), D^T (fp16 pairs)
 constexpr uint32_t COL_C1 = 0, COL_C3 = 256, COL_SP = 384, COL_DT = 448;
 constexpr uint32_t COL_P1 = 0, COL_W = 64;                                           // prep
+constexpr uint32_t COL_RB = 256;   // prep, sub-block path: one 64-column product per 16-row block
 constexpr uint32_t TMEM_COLS = 512;
+
+// ---- gate range. Per-token log-decays are floored at -10 (alpha >= e^-10 = 4.5e-5): a channel
+// that keeps less than that of its state per token has forgotten it to far below the precision
+// of the bf16 operands either way. A chunk takes the single-anchor path when, on every channel,
+// each 16-row quarter of the chunk decays by less than 2^-50 (so each half by less than
+// 2^-100, which keeps every anchored factor within 2^+-100); otherwise the sub-block path.
+constexpr float kFloorLog2 = -14.426950408889634f;   // log2(e^-10)
+constexpr float kQuarterRangeLog2 = 50.f;
 
 // ---- instruction descriptors (M = 128)
 constexpr uint32_t ID_P1 = idesc_f16(128, 64, 1, 1, 1);      // bf16, A MN-major, B MN-major
@@ -180,7 +200,11 @@ constexpr uint32_t ID_STATE_H = idesc_f16(128, 64, 1, 0, 1);   // the same, one 
 constexpr uint32_t ID_C3T = idesc_f16(128, 128, 0, 0, 0);      // fp16, A (D^T) in TMEM, B K-major
 constexpr uint32_t ID_OQK = idesc_f16(128, 64, 0, 0, 0);       // fp16, A (D^T) in TMEM, B (Aqk) K-major
 
+#ifdef KDA_TEST_HOOKS
+constexpr uint64_t kWaitLimitNs = 100000000ull;   // 100 ms in the test-only build
+#else
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+#endif
 
 struct TmaMaps {
     CUtensorMap q, k, g, v, o;
@@ -194,7 +218,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
         if (*abort_flag) return false;
         if (globaltimer() - t0 > kWaitLimitNs) {
             *abort_flag = 1;
-            atomicOr(&g_kda_device_error, 1u);
+            atomicOr(&g_kda_device_error, kErrTimeout);
             return false;
         }
     }
@@ -220,6 +244,20 @@ __device__ __forceinline__ float ex2_approx(float y) {
     float r;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y));
     return r;
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+    float r;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+constexpr float kLn2 = 0.6931471805599453f;
+
+// log2(sigmoid(x)) = min(x, 0) log2(e) - log2(1 + 2^(-|x| log2(e))), i.e. logsigmoid(x) in
+// log2 units, from the hardware 2^y and log2 approximations (absolute error about 1e-7)
+__device__ __forceinline__ float log2_sigmoid(float x) {
+    return fminf(x, 0.f) * kLog2e - lg2_approx(1.f + ex2_approx(-fabsf(x) * kLog2e));
 }
 
 // byte offset of 16-byte chunk j of row r in a tile of 128-byte rows, 128B swizzle
@@ -337,7 +375,7 @@ __device__ __forceinline__ bool wait_count(uint32_t addr, uint32_t target, volat
         if (*abort_flag) return false;
         if (globaltimer() - t0 > kWaitLimitNs) {
             *abort_flag = 1;
-            atomicOr(&g_kda_device_error, 1u);
+            atomicOr(&g_kda_device_error, kErrTimeout);
             return false;
         }
     }
@@ -355,7 +393,11 @@ __device__ __forceinline__ uint32_t smid() {
 // kRingPerCluster == true: `rings` holds one ring per cluster of this launch and
 // cluster c uses ring c (the allocation-free entry point, whose fixed scratch bounds
 // the cluster count).
-template <bool kRingPerCluster>
+// kGate: how g is given (kGateF32 / kGateBF16: log alpha per channel, fp32 or bf16 [rows, H, 128];
+// kGateScalar: one fp32 log alpha per token and head [rows, H], the same for every channel)
+// kNorm: q and k are L2-normalised per token and head first (the norms are applied in fp32 where
+// the operands are formed, so the normalised values are rounded only once)
+template <bool kRingPerCluster, int kGate, bool kNorm>
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_fwd_tc_kernel(const FwdParams p, const __grid_constant__ TmaMaps maps, unsigned char *rings) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -372,12 +414,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(miscg + M_ABORT);
 
     const int H = p.num_heads;
-    const int64_t unit = blockIdx.x / NS;
+    int64_t unit = blockIdx.x / NS;
+    // affine mode: units [0, N H) run each piece from a zero state, units [N H, 2 N H) from the
+    // identity with v = 0 (the piece's transition matrix); neither writes an output
+    const bool affine = p.mode == kModeAffine;
+    bool transition = false;
+    if (affine && unit >= static_cast<int64_t>(p.num_seqs) * p.num_heads) {
+        transition = true;
+        unit -= static_cast<int64_t>(p.num_seqs) * p.num_heads;
+    }
     const int h = static_cast<int>(unit % H);
     const int64_t s = unit / H;
     int64_t bos, eos;
-    if (p.cu_seqlens) {
+    bool cu_bad = false;
+    // segmented rows: unit s is segment j of row b, tokens [b T + j L, min(b T + (j + 1) L, (b + 1) T))
+    const int64_t seg_row = p.seg_len > 0 ? s / p.seg_count : s;
+    const int64_t seg_idx = p.seg_len > 0 ? s % p.seg_count : 0;
+    if (p.seg_len > 0) {
+        bos = seg_row * p.seq_len + seg_idx * p.seg_len;
+        const int64_t row_end = (seg_row + 1) * p.seq_len;
+        eos = bos + p.seg_len < row_end ? bos + p.seg_len : row_end;
+    } else if (p.cu_seqlens) {
         int64_t a = p.cu_seqlens[s], b = p.cu_seqlens[s + 1];
+        cu_bad = a < 0 || b < a || b > p.seq_len || (s == 0 && a != 0) || (s + 1 == p.num_seqs && b != p.seq_len);
         a = a < 0 ? 0 : (a > p.seq_len ? p.seq_len : a);
         b = b < 0 ? 0 : (b > p.seq_len ? p.seq_len : b);
         bos = a;
@@ -405,8 +464,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint32_t sm = smid();
             *reinterpret_cast<volatile uint32_t *>(miscg + M_SMID) = sm;
             *reinterpret_cast<volatile uint32_t *>(miscg + M_NEXT) = 0u;
-            *abort_flag = sm < static_cast<uint32_t>(kMaxRings) ? 0u : 1u;
-            if (sm >= static_cast<uint32_t>(kMaxRings)) atomicOr(&g_kda_device_error, 2u);
+            // the shared pool holds a ring per SM id; a launch with one ring per cluster does not
+            // index it by SM
+            const bool no_ring = !kRingPerCluster && sm >= static_cast<uint32_t>(kMaxRings);
+            *abort_flag = no_ring ? 1u : 0u;
+            if (no_ring) atomicOr(&g_kda_device_error, kErrRingIndex);
+            // a malformed cu_seqlens entry is reported (the sequence bounds were clamped above)
+            if (cu_bad) atomicOr(&g_kda_device_error, kErrCuSeqlens);
+            // where the final state goes: per unit, except that a segmented plain run writes only
+            // the last piece's, as its row's final state
+            void *const hT_ptr = transition ? p.hT_aux : p.hT;
+            const bool hT_write = hT_ptr != nullptr && (affine || p.seg_len == 0 || seg_idx == p.seg_count - 1);
+            *reinterpret_cast<void *volatile *>(miscg + M_HTINFO) = hT_ptr;
+            *reinterpret_cast<volatile size_t *>(miscg + M_HTINFO + 8) =
+                (!affine && p.seg_len > 0) ? (static_cast<size_t>(seg_row) * H + h) * D * D : state_base;
+            *reinterpret_cast<volatile uint32_t *>(miscg + M_HTINFO + 16) =
+                (hT_write ? 1u : 0u) | ((transition || p.hT_fp32 != 0) ? 2u : 0u);
         } else {
             for (int i = 0; i < PB_RING_FREE; ++i) mbar_init(BAR(i), i == PB_STAGE_FULL ? 2 : 1);
             *reinterpret_cast<volatile uint32_t *>(miscg + M_CONSUMED) = 0u;
@@ -454,7 +527,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int L = static_cast<int>(eos - t0 < C ? eos - t0 : C);
                 const uint32_t stage = sbase + CH_OST + sl * 16384;
                 if (!wait_bar(BAR(CB_O_READY), n & 1, abort_flag)) break;
-                if (L == C) {
+                if (affine) {
+                    // no output in affine mode
+                } else if (L == C) {
                     if (lane == 0) {
                         tma_store_3d(&maps.o, stage, 0, h, static_cast<int32_t>(t0));
                         tma_store_3d(&maps.o, stage + 8192, 64, h, static_cast<int32_t>(t0));
@@ -544,7 +619,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
             const int j0 = half * 64;                  // first key channel of this thread
             float S[64];
-            if (p.h0) {
+            if (transition) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) S[i] = (j0 + i == v) ? 1.f : 0.f;
+            } else if (p.h0 && !affine) {
                 if (p.h0_fp32) {
                     const float *src = static_cast<const float *>(p.h0) + state_base + v;
 #pragma unroll
@@ -720,14 +798,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (lane == 0) mbar_arrive(BAR(CB_O_READY));
                 }
             }
-            // final state: hT[j][v], coalesced across the warp for each key channel j
-            if (p.hT && !*abort_flag) {
-                if (p.hT_fp32) {
-                    float *dst = static_cast<float *>(p.hT) + state_base + v;
+            // final state: hT[j][v], coalesced across the warp for each key channel j (its place was
+            // noted in shared memory at setup, so that nothing of it stays live through the loop)
+            void *const hT_ptr = *reinterpret_cast<void *const volatile *>(miscg + M_HTINFO);
+            const size_t hT_base = *reinterpret_cast<const volatile size_t *>(miscg + M_HTINFO + 8);
+            const uint32_t hT_flags = *reinterpret_cast<const volatile uint32_t *>(miscg + M_HTINFO + 16);
+            const bool hT_fp32 = (hT_flags & 2u) != 0;
+            if ((hT_flags & 1u) && !*abort_flag) {
+                if (hT_fp32) {
+                    float *dst = static_cast<float *>(hT_ptr) + hT_base + v;
 #pragma unroll
                     for (int i = 0; i < 64; ++i) dst[static_cast<size_t>(j0 + i) * D] = S[i];
                 } else {
-                    uint16_t *dst = static_cast<uint16_t *>(p.hT) + state_base + v;
+                    uint16_t *dst = static_cast<uint16_t *>(hT_ptr) + hT_base + v;
 #pragma unroll
                     for (int i = 0; i < 64; ++i) dst[static_cast<size_t>(j0 + i) * D] = bf16_bits(S[i]);
                 }
@@ -760,23 +843,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int64_t t0 = bos + static_cast<int64_t>(m) * C;
                 const int32_t row = static_cast<int32_t>(t0);
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(BAR(PB_STAGE_FULL), STAGE_TX);
+                    mbar_arrive_expect_tx(BAR(PB_STAGE_FULL), kGate == kGateF32    ? STAGE_TX
+                                                              : kGate == kGateBF16 ? STAGE_TX - 16384u
+                                                                                   : STAGE_TX - 32768u);
                     tma_load_3d(sbase + PR_STG + STG_Q, &maps.q, BAR(PB_STAGE_FULL), 0, h, row);
                     tma_load_3d(sbase + PR_STG + STG_K, &maps.k, BAR(PB_STAGE_FULL), 0, h, row);
-                    tma_load_3d(sbase + PR_STG + STG_G, &maps.g, BAR(PB_STAGE_FULL), 0, h, row);
+                    // a bf16 gate tile goes to the upper half of the fp32 one's place
+                    if constexpr (kGate == kGateF32)
+                        tma_load_3d(sbase + PR_STG + STG_G, &maps.g, BAR(PB_STAGE_FULL), 0, h, row);
+                    else if constexpr (kGate == kGateBF16)
+                        tma_load_3d(sbase + PR_STG + STG_G + 16384, &maps.g, BAR(PB_STAGE_FULL), 0, h, row);
                 }
                 float *betaq = reinterpret_cast<float *>(miscg + M_BETAQ) + (kk & 1) * C;
                 for (int i = lane; i < C; i += 32) {
                     const int64_t tok = t0 + i;
                     betaq[i] = tok < eos ? p.beta[tok * H + h] : 0.f;
                 }
+                if constexpr (kGate == kGateScalar) {
+                    // one log alpha per token (activated here when asked); 0 past the end
+                    float *gq = reinterpret_cast<float *>(miscg + M_GSCALQ) + (kk & 1) * C;
+                    const float *gs = static_cast<const float *>(p.g);
+                    for (int i = lane; i < C; i += 32) {
+                        const int64_t tok = t0 + i;
+                        float x = tok < eos ? gs[tok * H + h] : 0.f;
+                        if ((p.flags & kFlagGateLogsigmoid) && tok < eos) x = log2_sigmoid(x) * kLn2;
+                        gq[i] = x;
+                    }
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(BAR(PB_STAGE_FULL));   // second arrival: index and beta stored
                 if (kk >= 1 && !wait_bar(BAR(PB_VSTAGE_FREE), (kk - 1) & 1, abort_flag)) break;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(BAR(PB_VSTAGE_FULL), VSTAGE_TX);
-                    tma_load_3d(sbase + PR_STG + STG_V, &maps.v, BAR(PB_VSTAGE_FULL), 0, h, row);
-                    tma_load_3d(sbase + PR_STG + STG_V + 8192, &maps.v, BAR(PB_VSTAGE_FULL), 64, h, row);
+                    if (transition) {
+                        mbar_arrive(BAR(PB_VSTAGE_FULL));   // v = 0: the tile was cleared once
+                    } else {
+                        mbar_arrive_expect_tx(BAR(PB_VSTAGE_FULL), VSTAGE_TX);
+                        tma_load_3d(sbase + PR_STG + STG_V, &maps.v, BAR(PB_VSTAGE_FULL), 0, h, row);
+                        tma_load_3d(sbase + PR_STG + STG_V + 8192, &maps.v, BAR(PB_VSTAGE_FULL), 64, h, row);
+                    }
                 }
                 __syncwarp();
             }
@@ -791,6 +895,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (m >= nch) break;
                 const int r = m % NRING;
                 unsigned char *set = ring + static_cast<uint64_t>(r) * SET_STRIDE;
+#ifdef KDA_TEST_HOOKS
+                if (m == g_kda_test_skip_chunk) {
+                    // hand the tiles back as if published, but never signal the ring slot
+                    if (lane == 0) {
+                        mbar_arrive(BAR(PB_OUTA_FREE));
+                        mbar_arrive(BAR(PB_VSTAGE_FREE));
+                    }
+                    __syncwarp();
+                    if (!wait_bar(BAR(PB_OUTB_READY), kk & 1, abort_flag)) break;
+                    if (!wait_bar(BAR(PB_OUTC_READY), kk & 1, abort_flag)) break;
+                    if (lane == 0) mbar_arrive(BAR(PB_OUTC_FREE));
+                    __syncwarp();
+                    continue;
+                }
+#endif
                 // the ring slot must have been pulled by the chain CTA (chunk m - NRING)
                 if (m >= NRING && !wait_count(misc + M_CONSUMED, static_cast<uint32_t>(m - NRING + 1), abort_flag))
                     break;
@@ -848,6 +967,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 st_shared_v4(sbase + PR_AVT + e * 16, 0u, 0u, 0u, 0u);   // rows 0..63 (T')
                 st_shared_v4(sbase + PR_TB + e * 16, 0u, 0u, 0u, 0u);
             }
+            if (transition) {
+                // v = 0 for a transition run: the value tile is never loaded; each thread clears the
+                // 16-byte pieces it converts every chunk
+#pragma unroll
+                for (int c2 = 0; c2 < 4; ++c2) st_shared_v4(sbase + PR_STG + STG_V + (t + 256 * c2) * 16, 0u, 0u, 0u, 0u);
+            }
             // A wait that gives up (abort) does not leave the loop on its own: the 8 warps leave
             // together at the next named barrier, which ORs the abort flag over them.
             for (int kk = 0;; ++kk) {
@@ -877,15 +1002,54 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             st_shared_v4(sbase + PR_STG + STG_Q + off, 0u, 0u, 0u, 0u);
                             st_shared_v4(sbase + PR_STG + STG_K + off, 0u, 0u, 0u, 0u);
                         }
-                        for (int e = t; e < (C - Lz) * 32; e += 256)
-                            st_shared_v4(sbase + PR_STG + STG_G + static_cast<uint32_t>((Lz + (e >> 5)) * 512 + (e & 31) * 16),
-                                         0u, 0u, 0u, 0u);
+                        if constexpr (kGate == kGateF32) {
+                            for (int e = t; e < (C - Lz) * 32; e += 256)
+                                st_shared_v4(sbase + PR_STG + STG_G +
+                                                 static_cast<uint32_t>((Lz + (e >> 5)) * 512 + (e & 31) * 16),
+                                             0u, 0u, 0u, 0u);
+                        } else if constexpr (kGate == kGateBF16) {
+                            for (int e = t; e < (C - Lz) * 16; e += 256)
+                                st_shared_v4(sbase + PR_STG + STG_G + 16384 +
+                                                 static_cast<uint32_t>((Lz + (e >> 4)) * 256 + (e & 15) * 16),
+                                             0u, 0u, 0u, 0u);
+                        }
                     }
                 }
                 if (named_bar_any(2, 256, no_chunk || *abort_flag != 0)) {
                     if (t == 0) mbar_arrive(BAR(PB_OUTA_READY));   // the publisher's end signal
                     break;
                 }
+                // rows of this chunk that hold tokens (the others are zero in the staging tiles)
+                const int Lrows = static_cast<int>(eos - (bos + static_cast<int64_t>(m) * C) < C
+                                                       ? eos - (bos + static_cast<int64_t>(m) * C)
+                                                       : C);
+                // 1 / ||x|| of each staged row of q (0..63) and k (64..127); a zero row gets a finite
+                // factor and stays zero
+                float *invn = reinterpret_cast<float *>(miscg + M_INVN);
+                if constexpr (kNorm) {
+#pragma unroll 1
+                    for (int rr = warp - 4; rr < 2 * C; rr += 8) {
+                        const uint32_t a = sbase + PR_STG + (rr < C ? STG_Q : STG_K) +
+                                           static_cast<uint32_t>((rr & (C - 1)) * 256 + lane * 8);
+                        uint32_t w0, w1;
+                        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(a) : "memory");
+                        const float x0 = lo_bf(w0), x1 = hi_bf(w0), x2 = lo_bf(w1), x3 = hi_bf(w1);
+                        float ss = x0 * x0 + x1 * x1 + x2 * x2 + x3 * x3;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                        if (lane == 0) invn[rr] = rsqrtf(fmaxf(ss, 1e-24f));
+                    }
+                    if (named_bar_any(2, 256, *abort_flag != 0)) break;
+                }
+                // a staged q / k element, normalised when asked
+                auto qn = [&](int r, float x) -> float {
+                    if constexpr (kNorm) return x * invn[r];
+                    return x;
+                };
+                auto kn = [&](int r, float x) -> float {
+                    if constexpr (kNorm) return x * invn[C + r];
+                    return x;
+                };
                 const float *beta_s = reinterpret_cast<const float *>(miscg + M_BETAQ) + (kk & 1) * C;
 #ifdef KDA_TRACE
                 if (t == 0 && blockIdx.x / 4 == KDA_TRACE_CLUSTER_ID && m < 64) {
@@ -904,6 +1068,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // were zeroed above.
                 uint32_t ktr[16];   // Kt^T of this thread: 4 fp16 pairs x 2 passes x 2 channels
                 const bool flip = (lane >> 2) & 1;
+                bool robust = false;   // this chunk takes the sub-block path (CTA-uniform)
                 {
                     const int grp = (warp - 4) & 3;
                     const int cp = grp * 16 + (lane & 15);
@@ -911,6 +1076,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const int c0 = 2 * cp, r0 = 16 * tq;
                     const int rp0 = r0 + (flip ? 8 : 0), rp1 = r0 + (flip ? 0 : 8);   // first row of each pass
                     const float *gst = reinterpret_cast<const float *>(sgen + PR_STG + STG_G);
+                    const uint32_t *gbf = reinterpret_cast<const uint32_t *>(sgen + PR_STG + STG_G + 16384);
+                    const float *gsc = reinterpret_cast<const float *>(miscg + M_GSCALQ) + (kk & 1) * C;
+                    const bool act = (p.flags & kFlagGateLogsigmoid) && kGate != kGateScalar;
                     const uint32_t *qst = reinterpret_cast<const uint32_t *>(sgen + PR_STG + STG_Q);
                     const uint32_t *kst = reinterpret_cast<const uint32_t *>(sgen + PR_STG + STG_K);
                     // g of the channel pair in log2 units (x, y = channels c0, c0 + 1), in pass order
@@ -920,18 +1088,80 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int rr = (i < 8 ? rp0 : rp1) + (i & 7);
-                        gv[i] = f2_mul(*reinterpret_cast<const float2 *>(gst + rr * D + c0), l2e);
+                        float2 gr;
+                        if constexpr (kGate == kGateF32) {
+                            gr = *reinterpret_cast<const float2 *>(gst + rr * D + c0);
+                        } else if constexpr (kGate == kGateBF16) {
+                            const uint32_t w = gbf[rr * (D / 2) + cp];
+                            gr = make_float2(lo_bf(w), hi_bf(w));
+                        } else {
+                            gr = make_float2(gsc[rr], gsc[rr]);
+                        }
+                        if (act) {
+                            // g holds the gate's pre-activation: log alpha = logsigmoid(g); rows past
+                            // the end of the sequence keep log alpha = 0
+                            gv[i] = rr < Lrows ? make_float2(log2_sigmoid(gr.x), log2_sigmoid(gr.y))
+                                               : make_float2(0.f, 0.f);
+                        } else {
+                            gv[i] = f2_mul(gr, l2e);
+                        }
+                        gv[i] = make_float2(fmaxf(gv[i].x, kFloorLog2), fmaxf(gv[i].y, kFloorLog2));
                         sp[i >> 3] = f2_add(sp[i >> 3], gv[i]);
                     }
                     // row-quarter sums of g per channel, [4][128] floats in the solve's scratch
                     float *gq = reinterpret_cast<float *>(sgen + PR_P);
-                    *reinterpret_cast<float2 *>(gq + tq * 128 + c0) = f2_add(sp[0], sp[1]);
-                    if (named_bar_any(2, 256, *abort_flag != 0)) break;
+                    const float2 qsum = f2_add(sp[0], sp[1]);
+                    *reinterpret_cast<float2 *>(gq + tq * 128 + c0) = qsum;
+                    // one barrier serves both the exchange and the choice of path: it ORs "this
+                    // quarter decays beyond the single anchor's range" with the abort flag; only when
+                    // that is set does a second barrier tell the two apart
+                    const bool unsafe = !(qsum.x >= -kQuarterRangeLog2) || !(qsum.y >= -kQuarterRangeLog2);
+                    if (named_bar_any(2, 256, unsafe || *abort_flag != 0)) {
+                        if (named_bar_any(2, 256, *abort_flag != 0)) break;
+                        robust = true;
+                    }
                     float2 qs[4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) qs[q] = *reinterpret_cast<const float2 *>(gq + q * 128 + c0);
                     const float2 ga = f2_add(qs[0], qs[1]);                  // G at the anchor row 31
                     const float2 gl = f2_add(ga, f2_add(qs[2], qs[3]));      // G at row 63
+                    if (robust) {
+                        // ---- sub-block path, part 1 (this thread's rows and channels): the running
+                        // log-decay G over the chunk, written over g in the staging tile for the factor
+                        // phase, Kt = K 2^(Gl - G) (<= 1), e^Gl; the anchored factors are not used.
+                        float2 run = make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int q = 0; q < 3; ++q)
+                            if (q < tq) run = f2_add(run, qs[q]);
+                        float *gstw = reinterpret_cast<float *>(sgen + PR_STG + STG_G);
+#pragma unroll
+                        for (int ps = 0; ps < 2; ++ps) {
+                            // pass 0 starts after the lower 8 rows when it is the upper half
+                            float2 Y = (ps == 0) == flip ? f2_add(run, sp[ps ^ 1]) : run;
+                            const int rb = ps == 0 ? rp0 : rp1;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                float2 kt[2];
+#pragma unroll
+                                for (int u = 0; u < 2; ++u) {
+                                    const int i = ps * 8 + 2 * e + u, rr = rb + 2 * e + u;
+                                    Y = f2_add(Y, gv[i]);
+                                    *reinterpret_cast<float2 *>(gstw + rr * D + c0) = Y;
+                                    const uint32_t kw = kst[rr * (D / 2) + cp];
+                                    kt[u] = f2_mul(make_float2(kn(rr, lo_bf(kw)), kn(rr, hi_bf(kw))),
+                                                   make_float2(ex2_approx(gl.x - Y.x), ex2_approx(gl.y - Y.y)));
+                                }
+                                ktr[ps * 4 + e] = pack_f16(kt[0].x, kt[1].x);
+                                ktr[8 + ps * 4 + e] = pack_f16(kt[0].y, kt[1].y);
+                            }
+                        }
+                        if (tq == 0) {
+                            *reinterpret_cast<float2 *>(dec_all + (kk & 1) * 128 + c0) =
+                                make_float2(ex2_approx(gl.x), ex2_approx(gl.y));
+                            // W and Qd are built from the chunk-start-relative factors directly
+                            *reinterpret_cast<float2 *>(ega_s + c0) = make_float2(1.f, 1.f);
+                        }
+                    } else {
                     // Y = G - Ga, running over a pass's rows; Y0 is its value before row r0
                     float2 Y0 = make_float2(-ga.x, -ga.y);
 #pragma unroll
@@ -957,8 +1187,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                 const float2 em = make_float2(ex2_approx(-Y.x), ex2_approx(-Y.y));
                                 const uint32_t kw = kst[rr * (D / 2) + cp];
                                 const uint32_t qw = qst[rr * (D / 2) + cp];
-                                const float2 k2 = make_float2(lo_bf(kw), hi_bf(kw));
-                                const float2 q2 = make_float2(lo_bf(qw), hi_bf(qw));
+                                const float2 k2 = make_float2(kn(rr, lo_bf(kw)), kn(rr, hi_bf(kw)));
+                                const float2 q2 = make_float2(qn(rr, lo_bf(qw)), qn(rr, hi_bf(qw)));
                                 kh[u] = f2_mul(k2, ep);
                                 qh[u] = f2_mul(q2, ep);
                                 kc[u] = f2_mul(k2, em);
@@ -988,18 +1218,86 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             make_float2(ex2_approx(gl.x), ex2_approx(gl.y));
                         *reinterpret_cast<float2 *>(ega_s + c0) = make_float2(ex2_approx(ga.x), ex2_approx(ga.y));
                     }
+                    }   // single-anchor path
+                }
+                if (robust) {
+                    // ---- sub-block path, part 2: the decayed blocks by 16-row block R, each with its own
+                    // anchor row a_R = 16R + 7:
+                    //   left  (A operand rows, all R):  [K; Q] 2^(G - G_aR)     rows of block R
+                    //   right (B operand of product R): K 2^(G_aR - G)          rows 0 .. 16R + 15, zero after
+                    // so that product R holds exactly the rows of block R of [Akk_raw; Aqk]. With the
+                    // floor, |G - G_aR| stays below 8 x 14.43 inside a block, and the right factor of an
+                    // earlier block is <= 1. The four right factors go to tiles that are dead until the
+                    // products have completed (Kt^T, A, T and the [T'; Aqk] tile), so the previous set's
+                    // part C must have been read out.
+                    if (named_bar_any(2, 256, *abort_flag != 0)) break;
+                    if (kk >= 1) wait_bar(BAR(PB_OUTC_FREE), (kk - 1) & 1, abort_flag);
+                    const int c = t & 127, hh = t >> 7;        // key channel, token half
+                    const float *G = reinterpret_cast<const float *>(sgen + PR_STG + STG_G);
+                    const uint16_t *kb = reinterpret_cast<const uint16_t *>(sgen + PR_STG + STG_K);
+                    const uint16_t *qb = reinterpret_cast<const uint16_t *>(sgen + PR_STG + STG_Q);
+                    float ganc[4];
+#pragma unroll
+                    for (int R = 0; R < 4; ++R) ganc[R] = G[(16 * R + 7) * D + c];
+                    const uint32_t right[4] = {sbase + PR_KC, sbase + PR_AKK, sbase + PR_T, sbase + PR_AVT};
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = 4 * hh + jj, R = j >> 1;   // 8-token group, its 16-row block
+                        float gg[8], kf[8], qf[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int r = 8 * j + e;
+                            gg[e] = G[r * D + c];
+                            kf[e] = kn(r, bf2f(kb[r * D + c]));
+                            qf[e] = qn(r, bf2f(qb[r * D + c]));
+                        }
+                        // anchor of this group's block, selected without a run-time index into ganc
+                        const float ga_own = (jj >> 1) ? (hh ? ganc[3] : ganc[1]) : (hh ? ganc[2] : ganc[0]);
+                        uint32_t kw[4], qw[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float f0 = ex2_approx(gg[2 * e] - ga_own), f1 = ex2_approx(gg[2 * e + 1] - ga_own);
+                            kw[e] = pack_bf16(kf[2 * e] * f0, kf[2 * e + 1] * f1);
+                            qw[e] = pack_bf16(qf[2 * e] * f0, qf[2 * e + 1] * f1);
+                        }
+                        st_shared_v4(sbase + PR_KH + sw128(c, j), kw[0], kw[1], kw[2], kw[3]);
+                        st_shared_v4(sbase + PR_QH + sw128(c, j), qw[0], qw[1], qw[2], qw[3]);
+#pragma unroll
+                        for (int Rp = 0; Rp < 4; ++Rp) {
+                            uint32_t w[4] = {0u, 0u, 0u, 0u};
+                            if (Rp >= R) {
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    w[e] = pack_bf16(kf[2 * e] * ex2_approx(ganc[Rp] - gg[2 * e]),
+                                                     kf[2 * e + 1] * ex2_approx(ganc[Rp] - gg[2 * e + 1]));
+                            }
+                            st_shared_v4(right[Rp] + sw128(c, j), w[0], w[1], w[2], w[3]);
+                        }
+                    }
                 }
                 fence_proxy_async_smem();
                 if (named_bar_any(2, 256, *abort_flag != 0)) break;
                 // The prep MMAs are issued by this thread right after the barrier that ends the
                 // phase writing their operands (no hop through another warp).
                 if (t == 0) {
-                    mbar_arrive(BAR(PB_STAGE_FREE));
                     tc_fence_after();
-                    // [Kh; Qh] Kc^T : A = Kh^T | Qh^T (MN-major, 64-row blocks 16 KB apart), B = Kc^T
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_f16(tmem + COL_P1, smem_desc(sbase + PR_KH + ks * 2048, 16384, 1024, kSwizzle128),
-                                smem_desc(sbase + PR_KC + ks * 2048, 16384, 1024, kSwizzle128), ID_P1, ks > 0);
+                    if (!robust) {
+                        mbar_arrive(BAR(PB_STAGE_FREE));
+                        // [Kh; Qh] Kc^T : A = Kh^T | Qh^T (MN-major, 64-row blocks 16 KB apart), B = Kc^T
+                        for (int ks = 0; ks < 8; ++ks)
+                            mma_f16(tmem + COL_P1, smem_desc(sbase + PR_KH + ks * 2048, 16384, 1024, kSwizzle128),
+                                    smem_desc(sbase + PR_KC + ks * 2048, 16384, 1024, kSwizzle128), ID_P1, ks > 0);
+                    } else {
+                        // the staging tile is still read after these products (G, q, k)
+#pragma unroll
+                        for (int R = 0; R < 4; ++R) {
+                            const uint32_t rt = sbase + (R == 0 ? PR_KC : R == 1 ? PR_AKK : R == 2 ? PR_T : PR_AVT);
+                            for (int ks = 0; ks < 8; ++ks)
+                                mma_f16(tmem + COL_RB + 64 * R,
+                                        smem_desc(sbase + PR_KH + ks * 2048, 16384, 1024, kSwizzle128),
+                                        smem_desc(rt + ks * 2048, 16384, 1024, kSwizzle128), ID_P1, ks > 0);
+                        }
+                    }
                     mma_commit(BAR(PB_P1_DONE));
                     KDA_TRACE_POINT(m, 2);
                 }
@@ -1032,8 +1330,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             }
                     }
                     uint32_t a[32];
-                    tmem_ld32(tmem + lane_base + COL_P1 + half * 32, a);
-                    tmem_wait_ld();
+                    if (!robust) {
+                        tmem_ld32(tmem + lane_base + COL_P1 + half * 32, a);
+                        tmem_wait_ld();
+                    } else {
+                        // row lrow belongs to block (lrow & 63) >> 4, whose product holds it: lanes 0-15 of
+                        // this warp read one product, lanes 16-31 the next
+                        const uint32_t col = COL_RB + 64u * static_cast<uint32_t>(2 * (q4 & 1)) + half * 32;
+                        uint32_t b[32];
+                        tmem_ld32(tmem + lane_base + col, a);
+                        tmem_ld32(tmem + lane_base + col + 64, b);
+                        tmem_wait_ld();
+                        if (lane >= 16) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) a[i] = b[i];
+                        }
+                    }
                     if (t == 0) KDA_TRACE_POINT(m, 27);
                     if (lrow < 64) {
                         const int rr = lrow;
@@ -1087,12 +1399,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         for (int r = 0; r < 16; ++r) T[(16 * wb + r) * AKK_LD + 16 * wb + li] = x[r];
                     }
                 }
+                if (robust) {
+                    // ---- sub-block path, part 3 (its products have completed): the W and Qd operands
+                    // from the chunk-start-relative factors, K 2^G and Q 2^G (<= 1), over the left factors
+                    // (the scale e^Ga applied to them later is 1 on this path); the T' rows of the
+                    // [T'; Aqk] tile held a right factor and must read as zero above the diagonal again
+                    const int c = t & 127, hh = t >> 7;
+                    const float *G = reinterpret_cast<const float *>(sgen + PR_STG + STG_G);
+                    const uint16_t *kb = reinterpret_cast<const uint16_t *>(sgen + PR_STG + STG_K);
+                    const uint16_t *qb = reinterpret_cast<const uint16_t *>(sgen + PR_STG + STG_Q);
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = 4 * hh + jj;
+                        uint32_t kw[4], qw[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int r = 8 * j + 2 * e;
+                            const float f0 = ex2_approx(G[r * D + c]), f1 = ex2_approx(G[(r + 1) * D + c]);
+                            kw[e] = pack_bf16(kn(r, bf2f(kb[r * D + c])) * f0, kn(r + 1, bf2f(kb[(r + 1) * D + c])) * f1);
+                            qw[e] = pack_bf16(qn(r, bf2f(qb[r * D + c])) * f0, qn(r + 1, bf2f(qb[(r + 1) * D + c])) * f1);
+                        }
+                        st_shared_v4(sbase + PR_KH + sw128(c, j), kw[0], kw[1], kw[2], kw[3]);
+                        st_shared_v4(sbase + PR_QH + sw128(c, j), qw[0], qw[1], qw[2], qw[3]);
+                    }
+                    for (int e = t; e < 512; e += 256) st_shared_v4(sbase + PR_AVT + e * 16, 0u, 0u, 0u, 0u);
+                }
                 if (t == 0) KDA_TRACE_POINT(m, 28);
                 fence_proxy_async_smem();
                 tc_fence_before();
                 if (named_bar_any(2, 256, *abort_flag != 0)) break;
                 if (t == 0) {
                     mbar_arrive(BAR(PB_OUTA_READY));
+                    if (robust) mbar_arrive(BAR(PB_STAGE_FREE));   // q, k and G have been read
                     KDA_TRACE_POINT(m, 9);
                 }
 
@@ -1332,20 +1670,48 @@ bool encode3d(CUtensorMap *map, const void *base, CUtensorMapDataType dt, uint32
     return r == CUDA_SUCCESS;
 }
 
-// Per-device ring pool of the operand-set exchange, allocated on first use and
-// held for the life of the process.
+// Per-device ring pool of the operand-set exchange, allocated on first use and held
+// until the library is unloaded (or the process exits).
 std::mutex g_pool_mu;
 unsigned char *g_pool[64] = {};
+bool g_exiting = false;
+void note_exit() { g_exiting = true; }
 
 unsigned char *ring_pool(int dev) {
     if (dev < 0 || dev >= 64) return nullptr;
     std::lock_guard<std::mutex> lk(g_pool_mu);
+    if (g_pool[dev]) {
+        // a device reset since the allocation frees the pool: allocate it again
+        cudaPointerAttributes at;
+        if (cudaPointerGetAttributes(&at, g_pool[dev]) != cudaSuccess || at.type != cudaMemoryTypeDevice) {
+            (void)cudaGetLastError();
+            g_pool[dev] = nullptr;
+        }
+    }
     if (!g_pool[dev]) {
         void *ptr = nullptr;
         if (cudaMalloc(&ptr, static_cast<size_t>(tc::kMaxRings) * tc::RING_BYTES) != cudaSuccess) return nullptr;
         g_pool[dev] = static_cast<unsigned char *>(ptr);
+        static std::once_flag once;
+        std::call_once(once, [] { std::atexit(note_exit); });
     }
     return g_pool[dev];
+}
+
+// Release the pools when the library is unloaded before the process exits. At exit
+// nothing is called: the CUDA runtime may already be torn down, and the driver reclaims
+// the memory with the process.
+__attribute__((destructor)) void release_ring_pools() {
+    if (g_exiting) return;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return;
+    for (int dev = 0; dev < 64; ++dev) {
+        if (!g_pool[dev]) continue;
+        if (cudaSetDevice(dev) == cudaSuccess) (void)cudaFree(g_pool[dev]);
+        g_pool[dev] = nullptr;
+    }
+    (void)cudaSetDevice(cur);
+    (void)cudaGetLastError();
 }
 
 // Scratch of the allocation-free entry point: one operand-set ring per cluster for at
@@ -1373,7 +1739,7 @@ cudaError_t noalloc_scratch(int dev, unsigned char **out) {
 }
 
 // Encode the tensor maps and launch one 4-CTA cluster per (sequence, head).
-template <bool kRingPerCluster>
+template <bool kRingPerCluster, int kGate, bool kNorm>
 cudaError_t launch_clusters(const FwdParams &p, int64_t rows, int64_t grid, unsigned char *rings,
                             cudaStream_t stream) {
     tc::TmaMaps maps;
@@ -1384,15 +1750,17 @@ cudaError_t launch_clusters(const FwdParams &p, int64_t rows, int64_t grid, unsi
                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
             !encode3d(&maps.k, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.num_heads, rows, 128,
                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
-            !encode3d(&maps.g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.num_heads, rows, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            (kGate == kGateF32 && !encode3d(&maps.g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.num_heads,
+                                            rows, 128, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
+            (kGate == kGateBF16 && !encode3d(&maps.g, p.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.num_heads,
+                                             rows, 128, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
             !encode3d(&maps.v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.num_heads, rows, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
             !encode3d(&maps.o, p.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.num_heads, rows, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
-    cudaError_t err = cudaFuncSetAttribute(tc::kda_fwd_tc_kernel<kRingPerCluster>,
+    cudaError_t err = cudaFuncSetAttribute(tc::kda_fwd_tc_kernel<kRingPerCluster, kGate, kNorm>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(tc::SMEM_BYTES));
     if (err != cudaSuccess) return err;
@@ -1408,7 +1776,7 @@ cudaError_t launch_clusters(const FwdParams &p, int64_t rows, int64_t grid, unsi
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, tc::kda_fwd_tc_kernel<kRingPerCluster>, p, maps, rings);
+    err = cudaLaunchKernelEx(&cfg, tc::kda_fwd_tc_kernel<kRingPerCluster, kGate, kNorm>, p, maps, rings);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
@@ -1416,7 +1784,7 @@ cudaError_t launch_clusters(const FwdParams &p, int64_t rows, int64_t grid, unsi
 }  // namespace
 
 cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream) {
-    const int64_t units = static_cast<int64_t>(p.num_seqs) * p.num_heads;
+    const int64_t units = static_cast<int64_t>(p.num_seqs) * p.num_heads * (p.mode == kModeAffine ? 2 : 1);
     if (units == 0) return cudaSuccess;
     const int64_t grid = units * tc::NS;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
@@ -1425,7 +1793,19 @@ cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream)
     if (err != cudaSuccess) return err;
     unsigned char *rings = ring_pool(dev);
     if (!rings) return cudaErrorMemoryAllocation;
-    return launch_clusters<false>(p, rows, grid, rings, stream);
+    const bool norm = (p.flags & kFlagL2NormQK) != 0;
+    switch (p.gate_mode) {
+        case kGateF32:
+            return norm ? launch_clusters<false, kGateF32, true>(p, rows, grid, rings, stream)
+                        : launch_clusters<false, kGateF32, false>(p, rows, grid, rings, stream);
+        case kGateBF16:
+            return norm ? launch_clusters<false, kGateBF16, true>(p, rows, grid, rings, stream)
+                        : launch_clusters<false, kGateBF16, false>(p, rows, grid, rings, stream);
+        case kGateScalar:
+            return norm ? launch_clusters<false, kGateScalar, true>(p, rows, grid, rings, stream)
+                        : launch_clusters<false, kGateScalar, false>(p, rows, grid, rings, stream);
+    }
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_fwd_tc_noalloc(const FwdParams &p, int64_t rows, cudaStream_t stream) {
@@ -1438,8 +1818,15 @@ cudaError_t launch_fwd_tc_noalloc(const FwdParams &p, int64_t rows, cudaStream_t
     unsigned char *rings = nullptr;
     err = noalloc_scratch(dev, &rings);
     if (err != cudaSuccess) return err;
-    return launch_clusters<true>(p, rows, units * tc::NS, rings, stream);
+    if (p.gate_mode != kGateF32 || p.flags != 0) return cudaErrorInvalidValue;
+    return launch_clusters<true, kGateF32, false>(p, rows, units * tc::NS, rings, stream);
 }
+
+#ifdef KDA_TEST_HOOKS
+extern "C" int kda_test_set_skip_chunk(int chunk) {
+    return static_cast<int>(cudaMemcpyToSymbol(g_kda_test_skip_chunk, &chunk, sizeof(int)));
+}
+#endif
 
 #ifdef KDA_TRACE
 extern "C" int kda_trace_read(unsigned long long *host) {

@@ -59,7 +59,21 @@ def run_oracle(inp: dict, heads=None, prefix=None):
     return oracle.kda_oracle(q, k, v, g, beta, inp["scale"], h0=h0)
 
 
-def check(inp, out_gpu, hT_gpu, heads=None, prefix=None, state=True, out_tol=OUT_TOL):
+def record(r_out, r_state, note=""):
+    """Print the measured errors and, when KDA_PARITY_LOG names a file, append them to it
+    (one line per check: test id, out error, state error), so that a run keeps its margins."""
+    import os
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    st = "-" if r_state is None else f"{r_state:.3e}"
+    line = f"{test}{(' ' + note) if note else ''}\tout {r_out:.3e}\tstate {st}"
+    print(line)
+    path = os.environ.get("KDA_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(line + "\n")
+
+
+def check(inp, out_gpu, hT_gpu, heads=None, prefix=None, state=True, out_tol=OUT_TOL, note=""):
     eo, eh = run_oracle(inp, heads=heads, prefix=prefix)
     og = out_gpu
     if heads is not None:
@@ -73,6 +87,9 @@ def check(inp, out_gpu, hT_gpu, heads=None, prefix=None, state=True, out_tol=OUT
         hg = hT_gpu if heads is None else hT_gpu[:, heads]
         hg = hg.float().cpu().numpy()
         r_state = rel(hg, eh)
+    record(r_out, r_state, note)
+    if r_state is not None:
         assert r_state <= STATE_TOL[hT_gpu.dtype], f"state rel err {r_state:.3e}"
+    assert np.isfinite(og).all(), "non-finite output"
     assert r_out <= out_tol, f"out rel err {r_out:.3e}"
     return r_out, r_state

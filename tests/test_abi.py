@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for st in range(0, 12):
+    for st in range(0, 16):
         s = kda.status_string(st)
         assert s.startswith("KDA_"), s
     assert kda.status_string(1234) == "KDA_ERR_UNKNOWN"
@@ -117,3 +117,72 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         kda.kda_fwd(x, x, x, x.float(), torch.zeros(1, 64, 1))
+
+
+def _fwd_args():
+    import torch
+    B, T, H = 1, 64, 2
+    q = torch.zeros(B, T, H, 128, dtype=torch.bfloat16)
+    return dict(q=q, k=q.clone(), v=q.clone(), g=torch.zeros(B, T, H, 128), beta=torch.zeros(B, T, H))
+
+
+@pytest.mark.parametrize("name,bad", [
+    ("out", lambda t: t.zeros(1, 63, 2, 128, dtype=t.bfloat16)),
+    ("initial_state", lambda t: t.zeros(1, 2, 128, 127)),
+    ("final_state", lambda t: t.zeros(2, 2, 128, 128)),
+    ("v", lambda t: t.zeros(1, 65, 2, 128, dtype=t.bfloat16)),
+    ("beta", lambda t: t.zeros(1, 64, 3)),
+])
+def test_binding_requires_exact_buffer_shapes(name, bad):
+    """An undersized buffer would be written out of bounds through the C ABI, which
+    sees only pointers: the binding refuses it before anything else."""
+    import torch
+    a = _fwd_args()
+    kw = {}
+    if name in a:
+        a[name] = bad(torch)
+    else:
+        kw[name] = bad(torch)
+    with pytest.raises(ValueError, match="shape"):
+        kda.kda_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], **kw)
+
+
+def test_binding_requires_exact_decode_shapes():
+    import torch
+    q = torch.zeros(4, 2, 128, dtype=torch.bfloat16)
+    g, beta = torch.zeros(4, 2, 128), torch.zeros(4, 2)
+    with pytest.raises(ValueError, match="shape"):
+        kda.kda_decode(q, q, q, g, beta, state_in=torch.zeros(4, 2, 128, 64))
+    with pytest.raises(ValueError, match="shape"):
+        kda.kda_decode(q, q, q, g, beta, out=torch.zeros(3, 2, 128, dtype=torch.bfloat16))
+
+
+def call_ex(lib, kind=0, flags=0, g=FAKE, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, beta=FAKE, out=FAKE)
+    a.update(kw)
+    return lib.kda_fwd_ex(a["q"], a["k"], a["v"], g, kind, a["beta"], 1.0, None, 0, 1, 64, 2, 128, 128,
+                          None, 0, None, 0, a["out"], flags, None)
+
+
+def test_fwd_ex_rejects_unknown_options(lib):
+    KDA_ERR_BAD_OPTION = 14
+    assert call_ex(lib, kind=3) == KDA_ERR_BAD_OPTION
+    assert call_ex(lib, kind=-1) == KDA_ERR_BAD_OPTION
+    assert call_ex(lib, flags=4) == KDA_ERR_BAD_OPTION
+    assert kda.status_string(KDA_ERR_BAD_OPTION).startswith("KDA_ERR_BAD_OPTION")
+
+
+def test_fwd_ex_gate_alignment(lib):
+    # a per-channel gate is loaded by TMA (16 bytes); a per-token one needs only 4
+    assert call_ex(lib, kind=1, g=ctypes.c_void_p(0x10004)) == 7
+    assert call_ex(lib, kind=2, g=ctypes.c_void_p(0x10002)) == 7
+    import torch
+    if not torch.cuda.is_available():
+        assert call_ex(lib, kind=2, g=ctypes.c_void_p(0x10004), flags=3) == 5   # passes; no device
+
+
+def test_segmented_workspace_size(lib):
+    f = lib.kda_fwd_segmented_workspace
+    assert f(1, 1 << 20, 32, 1 << 15) == 3 * 32 * 32 * 128 * 128 * 4
+    assert f(2, 1000, 3, 192) == 3 * 2 * 6 * 3 * 128 * 128 * 4
+    assert f(1, 1000, 3, 100) == 0 and f(1, 1000, 3, 0) == 0 and f(1, 1000, 0, 64) == 0

@@ -133,6 +133,61 @@ def test_strong_decay():
     check(inp, out, hT)
 
 
+# -- the whole gate range: any log alpha <= 0 ------------------------------------
+# Chunks in which some channel decays by more than 2^-100 over half a chunk take the
+# sub-block path; these cases put every chunk, or some chunks, there.
+
+@pytest.mark.parametrize("mu", [-3.0, -6.0])
+def test_very_strong_decay_every_chunk(mu):
+    # logsigmoid(N(-3, 1)) is about -3 per token: about -200 over 64 tokens;
+    # logsigmoid(N(-6, 1)) about -6 per token
+    inp = gpu_inputs("t4k_h32", T=650, H=2, g_mu=mu)
+    out, hT = run_gpu(inp)
+    check(inp, out, hT, note=f"g=logsigmoid(N({mu},1))")
+
+
+def test_one_channel_at_minus_20_per_token():
+    inp = gpu_inputs("t4k_h32", T=650, H=3)
+    inp["g"][..., 5] = -20.0
+    out, hT = run_gpu(inp)
+    check(inp, out, hT)
+
+
+def test_zero_alpha_tokens():
+    # alpha = 0 (g = -inf) on a run of tokens and channels: the state forgets those channels
+    inp = gpu_inputs("t4k_h32", T=400, H=2)
+    inp["g"][:, 100:140, :, 7:40] = float("-inf")
+    out, hT = run_gpu(inp)
+    check(inp, out, hT)
+
+
+def test_strong_decay_in_some_chunks_only():
+    # ordinary gates with bursts of fast decay: neighbouring chunks take different paths
+    # inside one (sequence, head), on ragged varlen sequences
+    inp = varlen_case([700, 130, 0, 321], H=3)
+    g = inp["g"]
+    for t0, t1 in [(70, 140), (300, 330), (700 + 30, 700 + 100), (830 + 250, 830 + 321)]:
+        g[:, t0:t1, 1:, ::3] = -12.0
+    out, hT = run_gpu(inp)
+    check(inp, out, hT)
+
+
+def test_malformed_cu_seqlens_is_reported():
+    """A cu_seqlens table that does not run 0, ..., T without decreasing is detected on the
+    device and reported by kda_device_error; the device keeps working afterwards."""
+    import kimi_delta_attention_27_b200 as kda
+    KDA_ERR_BAD_CU_SEQLENS = 12
+    inp = varlen_case([100, 90, 60], H=2)
+    assert kda.device_error() == 0
+    for table in ([0, 100, 50, 250], [3, 100, 190, 250], [0, 100, 190, 240]):
+        bad = dict(inp, cu_seqlens=torch.tensor(table, dtype=torch.int32, device="cuda"))
+        run_gpu(bad)
+        assert kda.device_error() == KDA_ERR_BAD_CU_SEQLENS, table
+    out, hT = run_gpu(inp)
+    assert kda.device_error() == 0
+    check(inp, out, hT)
+
+
 def test_split_call_resume_matches_single_call():
     inp = gpu_inputs("t4k_h32", T=1000, H=4)
     out, hT = run_gpu(inp)
