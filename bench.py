@@ -12,9 +12,12 @@ C = 64, fp32 final state), inputs resident in HBM before the timed region
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                   [--workload NAME] [--no-cpu-baseline] [--no-e2e]
 
-Prints ONE JSON line on rank 0. Multi-GPU runs (torchrun, one rank per GPU)
-give each rank its own independent workload (weak scaling, no collective on
-the data path; NCCL only for the barrier and the max-over-ranks time).
+Prints ONE JSON line on rank 0. Multi-GPU runs (torchrun, one rank per GPU;
+``--gpus N`` without torchrun starts the N ranks itself) give each rank its own
+independent workload (weak scaling), or with ``--split heads`` share one
+workload's heads between the ranks (strong scaling). Either way there is no
+collective on the data path: NCCL carries only the barrier and the
+max-over-ranks time.
 """
 from __future__ import annotations
 
@@ -186,9 +189,29 @@ def rank_seed(base_seed: int, rank: int) -> int:
     return base_seed + 1000 * rank
 
 
+def head_range(H: int, world: int, rank: int) -> tuple[int, int]:
+    """Heads [h0, h1) of rank ``rank`` when ``world`` ranks share H heads (strong scaling):
+    contiguous blocks, the first H % world ranks one head more."""
+    base, extra = divmod(H, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
+
+
+def take_heads(inp: dict, h0: int, h1: int) -> dict:
+    """The workload restricted to heads [h0, h1) (contiguous copies)."""
+    d = dict(inp)
+    for key in ("q", "k", "v", "g", "beta"):
+        d[key] = inp[key][:, :, h0:h1].contiguous()
+    if inp["h0"] is not None:
+        d["h0"] = inp["h0"][:, h0:h1].contiguous()
+    d["H"] = h1 - h0
+    return d
+
+
 def cpu_baseline_run(inp, tokens_per_step, steps=1, warmup=0):
     """Time the fp64 oracle, as it stands, on the host cores over the first
-    ``tokens_per_step`` tokens of the workload (all heads)."""
+    ``tokens_per_step`` tokens of the workload (all heads). The last run's output
+    is returned too (``out``), so that the timed GPU output can be compared with it."""
     import oracle
     sample = {}
     for name in ("q", "k", "v", "g", "beta"):
@@ -196,16 +219,33 @@ def cpu_baseline_run(inp, tokens_per_step, steps=1, warmup=0):
     h0 = None if inp["h0"] is None else inp["h0"][:1].cpu().double()
     threads = os.cpu_count() or 1
     times = []
+    eo = None
     for i in range(warmup + steps):
         t = time.perf_counter()
-        oracle.kda_oracle(sample["q"], sample["k"], sample["v"], sample["g"], sample["beta"],
-                          inp["scale"], h0=h0, nthreads=threads)
+        eo, _ = oracle.kda_oracle(sample["q"], sample["k"], sample["v"], sample["g"], sample["beta"],
+                                  inp["scale"], h0=h0, nthreads=threads)
         dt = time.perf_counter() - t
         if i >= warmup:
             times.append(dt)
     H = inp["H"]
     used = min(threads, H)  # the oracle runs one (sequence, head) unit per thread
-    return dict(seconds=times, tokens=tokens_per_step, heads=H, threads=used)
+    return dict(seconds=times, tokens=tokens_per_step, heads=H, threads=used, out=eo)
+
+
+def parity_of_sample(out_gpu, inp, r) -> dict:
+    """max|d out| / max|out| of the timed GPU output against the CPU-baseline oracle run
+    ``r`` (the first tokens of row 0, all heads; for a packed batch only the tokens of
+    its first sequence, where the oracle's single-sequence sample is the same problem)."""
+    import numpy as np
+    n = r["tokens"]
+    if inp["cu_seqlens"] is not None:
+        n = min(n, int(inp["lengths"][0]))
+    ref = np.asarray(r["out"])[:, :n]
+    got = out_gpu[:1, :n].float().cpu().numpy()
+    err = float(np.abs(got - ref).max() / max(float(np.abs(ref).max()), 1e-30))
+    return {"out_rel_err": err, "bar": 1e-2, "tokens": n, "heads": r["heads"],
+            "sample": f"first {n} tokens of row 0, every head, against the fp64 oracle "
+                      "(the CPU-baseline run)"}
 
 
 def reference_arm(args, world, rank):
@@ -249,13 +289,16 @@ WORKLOAD_TEXT = {
 }
 
 
-def workload_config(name, world, note=None):
+def workload_config(name, world, note=None, split="none"):
     from kimi_delta_attention_27_b200.inputs import CONFIGS
     c = CONFIGS[name]
+    strong = split == "heads"
+    per = c["B"] if c.get("lengths") is None else c["lengths"][0]
     cfg = {"workload": WORKLOAD_TEXT.get(name, name), "name": name,
-           "global_batch": (c["B"] if c.get("lengths") is None else c["lengths"][0]) * world,
+           "global_batch": per if strong else per * world,
            "seq_len": c["T"], "heads": c["H"], "head_dim": D, "chunk": C,
-           "parallelism": f"dp{world}" if world > 1 else "single-gpu",
+           "parallelism": (f"heads split over {world} ranks" if strong else f"dp{world}") if world > 1
+           else "single-gpu",
            "l2": "inputs larger than L2 (no flush needed)"}
     if note:
         cfg["note"] = note
@@ -277,6 +320,9 @@ def main():
                     help="tokens (all heads) per reference-arm step")
     ap.add_argument("--e2e-slice", type=int, default=1 << 16,
                     help="tokens per host->device slice in the end-to-end measurement")
+    ap.add_argument("--split", default="none", choices=["none", "heads"],
+                    help="none: each rank runs its own copy of the workload (weak scaling); "
+                         "heads: the ranks share the workload's heads (strong scaling)")
     ap.add_argument("--decode", default=None, metavar="BxH[:bf16]",
                     help="time the single-token decode step instead (e.g. 256x32 or 256x32:bf16); "
                          "prints its own line, not the prefill metric")
@@ -285,8 +331,15 @@ def main():
     if args.decode:
         return decode_main(args)
 
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch_under_torchrun(args.gpus)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if world != args.gpus:
+        if rank == 0:
+            print(f"bench.py: --gpus {args.gpus} but {world} ranks were started; no line printed",
+                  file=sys.stderr)
+        return 2
     if args.impl == "reference":
         return reference_arm(args, world, rank)
 
@@ -297,7 +350,18 @@ def main():
 
     name = args.workload
     cfg = dict(CONFIGS[name])
-    inp = make_inputs(name, device="cuda", seed=rank_seed(cfg["seed"], rank))
+    strong = args.split == "heads"
+    if strong:
+        # one workload (the same seed on every rank), this rank's heads of it
+        full = make_inputs(name, device="cuda")
+        h_lo, h_hi = head_range(full["H"], world, rank)
+        inp = take_heads(full, h_lo, h_hi)
+        H_all = full["H"]
+        del full
+        torch.cuda.empty_cache()
+    else:
+        inp = make_inputs(name, device="cuda", seed=rank_seed(cfg["seed"], rank))
+        H_all = inp["H"]
     H, N, tokens = inp["H"], inp["N"], inp["B"] * inp["T"]
     final_dt = inp["final_dtype"]
     out = torch.empty_like(inp["v"])
@@ -336,8 +400,9 @@ def main():
     total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
     launch_ms = [a.elapsed_time(b) for a, b in ev]
     ms_per_step = total_ms / args.steps
-    value = whole_job_value(world, tokens, ms_per_step)
-    flops = pages_flops(tokens, H)
+    # weak: every rank processed its own tokens; strong: the ranks shared one workload's tokens
+    value = (tokens / (ms_per_step / 1e3)) if strong else whole_job_value(world, tokens, ms_per_step)
+    flops = pages_flops(tokens, H_all) if strong else world * pages_flops(tokens, H)
     peaks = load_peaks()
     alg_bytes = tokens * H * BYTES_PER_TOKEN_HEAD + state_bytes(
         N, H, None if inp["h0"] is None else inp["h0"].dtype, final_dt)
@@ -348,9 +413,10 @@ def main():
     # ---- end to end: pinned host buffers -> device -> kda_fwd -> host, per step
     e2e = None
     if not args.no_e2e:
-        e2e = e2e_run(args, inp, world, rank)
+        e2e = e2e_run(args, inp, world, rank, strong=strong)
 
     cpu = None
+    parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # size the sample for roughly 10-30 s of host work: probe, then scale up
         ntok = min(args.cpu_tokens, tokens)
@@ -365,23 +431,25 @@ def main():
                "kind": "oracle",
                "sample": f"first {r['tokens']} tokens of all {r['heads']} heads of the workload "
                          f"({secs:.1f} s, {os.cpu_count()} host cores, one thread per head)"}
+        parity = parity_of_sample(out, inp, r)
 
     del inp
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": workload_config(name, world),
-            "tflops": world * flops / (ms_per_step / 1e3) / 1e12,
-            "frac_bf16_peak": world * flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"] / world,
+            "higher_is_better": True, "scaling": "strong" if strong else "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(name, world, split=args.split),
+            "tflops": flops / (ms_per_step / 1e3) / 1e12,
+            "frac_bf16_peak": flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"] / world,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
                          "traffic": traffic, "peak_source": peaks["source"],
                          "kernel": prof_kernel or "kda_fwd",
                          "alg_bytes_per_launch": alg_bytes,
                          "avg_launch_ms": avg_launch_s * 1e3},
-            "cpu_baseline": cpu, "e2e": e2e,
+            "cpu_baseline": cpu, "e2e": e2e, "parity": parity,
             "gpu_launches": args.steps * 1,
             "clocks": clocks,
         }
@@ -469,7 +537,20 @@ def decode_main(args):
     return 0
 
 
-def e2e_run(args, inp, world, rank):
+def relaunch_under_torchrun(n: int) -> int:
+    """``--gpus N`` started without torchrun: run this command again as N ranks (one per
+    GPU, rendezvous on 127.0.0.1) and return their exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__),
+           *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def e2e_run(args, inp, world, rank, strong=False):
     """Same metric through the public API with host buffers: every step streams
     the whole sequence through the device in slices (chunked prefill, state
     carried between slices), copying each slice's inputs host->device from
@@ -538,12 +619,14 @@ def e2e_run(args, inp, world, rank):
     t1.record(comp_s)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1), world) / steps
-    return {"value": world * nsl * Ls / (ms / 1e3), "unit": "tokens/s",
+    return {"value": (1 if strong else world) * nsl * Ls / (ms / 1e3), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "steps": steps, "slice_tokens": Ls,
             "how": "public binding kda_fwd over the sequence in slices with state carry; "
                    "pinned host inputs copied per slice on a copy stream (double-buffered), "
-                   "output copied back per slice"}
+                   "output copied back per slice. The host holds one slice of the workload's "
+                   "synthetic inputs and streams it for every slice: the bytes copied and the work "
+                   "per slice are the full sequence's, the values are not the workload's own"}
 
 
 if __name__ == "__main__":

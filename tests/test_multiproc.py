@@ -83,3 +83,41 @@ def test_whole_job_value_counts_every_rank():
     assert bench.whole_job_value(4, 1 << 20, 50.0) == pytest.approx(83886080.0)
     assert bench.whole_job_value(1, 1 << 20, 50.0) == pytest.approx(20971520.0)
     assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def test_gpus_flag_starts_that_many_ranks(tmp_path):
+    """``bench.py --gpus 2`` without torchrun starts two ranks itself (torchrun on
+    127.0.0.1) and prints one line, for two GPUs; here through the reference arm, which
+    runs on the host cores (rank 0 works, rank 1 exits at once)."""
+    import json
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "3", "--workload", "t256_h1",
+                        "--ref-tokens", "64"],
+                       env=env, capture_output=True, text=True, timeout=300, cwd=str(tmp_path))
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    assert json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_rank_count_must_match_gpus_flag(tmp_path):
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "3"],
+                       env=env, capture_output=True, text=True, timeout=120, cwd=str(tmp_path))
+    assert r.returncode == 2
+    assert r.stdout.strip() == ""
+
+
+def test_head_split_covers_every_head_once():
+    import bench
+    for H, world in [(32, 8), (32, 3), (5, 4), (1, 1), (32, 32)]:
+        seen = []
+        for rank in range(world):
+            h0, h1 = bench.head_range(H, world, rank)
+            assert 0 <= h0 <= h1 <= H
+            seen += list(range(h0, h1))
+        assert seen == list(range(H))
+        sizes = [bench.head_range(H, world, r)[1] - bench.head_range(H, world, r)[0] for r in range(world)]
+        assert max(sizes) - min(sizes) <= 1
