@@ -397,7 +397,9 @@ __device__ __forceinline__ uint32_t smid() {
 // kGateScalar: one fp32 log alpha per token and head [rows, H], the same for every channel)
 // kNorm: q and k are L2-normalised per token and head first (the norms are applied in fp32 where
 // the operands are formed, so the normalised values are rounded only once)
-template <bool kRingPerCluster, int kGate, bool kNorm>
+// kSeg: the launch may be segmented or affine (FwdParams::seg_len, mode); other launches compile
+// none of that bookkeeping
+template <bool kRingPerCluster, int kGate, bool kNorm, bool kSeg>
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_fwd_tc_kernel(const FwdParams p, const __grid_constant__ TmaMaps maps, unsigned char *rings) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -417,7 +419,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int64_t unit = blockIdx.x / NS;
     // affine mode: units [0, N H) run each piece from a zero state, units [N H, 2 N H) from the
     // identity with v = 0 (the piece's transition matrix); neither writes an output
-    const bool affine = p.mode == kModeAffine;
+    const bool affine = kSeg && p.mode == kModeAffine;
     bool transition = false;
     if (affine && unit >= static_cast<int64_t>(p.num_seqs) * p.num_heads) {
         transition = true;
@@ -428,9 +430,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int64_t bos, eos;
     bool cu_bad = false;
     // segmented rows: unit s is segment j of row b, tokens [b T + j L, min(b T + (j + 1) L, (b + 1) T))
-    const int64_t seg_row = p.seg_len > 0 ? s / p.seg_count : s;
-    const int64_t seg_idx = p.seg_len > 0 ? s % p.seg_count : 0;
-    if (p.seg_len > 0) {
+    const bool segmented = kSeg && p.seg_len > 0;
+    const int64_t seg_row = segmented ? s / p.seg_count : s;
+    const int64_t seg_idx = segmented ? s % p.seg_count : 0;
+    if (segmented) {
         bos = seg_row * p.seq_len + seg_idx * p.seg_len;
         const int64_t row_end = (seg_row + 1) * p.seq_len;
         eos = bos + p.seg_len < row_end ? bos + p.seg_len : row_end;
@@ -474,10 +477,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // where the final state goes: per unit, except that a segmented plain run writes only
             // the last piece's, as its row's final state
             void *const hT_ptr = transition ? p.hT_aux : p.hT;
-            const bool hT_write = hT_ptr != nullptr && (affine || p.seg_len == 0 || seg_idx == p.seg_count - 1);
+            const bool hT_write = hT_ptr != nullptr && (affine || !segmented || seg_idx == p.seg_count - 1);
             *reinterpret_cast<void *volatile *>(miscg + M_HTINFO) = hT_ptr;
             *reinterpret_cast<volatile size_t *>(miscg + M_HTINFO + 8) =
-                (!affine && p.seg_len > 0) ? (static_cast<size_t>(seg_row) * H + h) * D * D : state_base;
+                (!affine && segmented) ? (static_cast<size_t>(seg_row) * H + h) * D * D : state_base;
             *reinterpret_cast<volatile uint32_t *>(miscg + M_HTINFO + 16) =
                 (hT_write ? 1u : 0u) | ((transition || p.hT_fp32 != 0) ? 2u : 0u);
         } else {
@@ -1088,26 +1091,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int rr = (i < 8 ? rp0 : rp1) + (i & 7);
-                        float2 gr;
                         if constexpr (kGate == kGateF32) {
-                            gr = *reinterpret_cast<const float2 *>(gst + rr * D + c0);
+                            gv[i] = *reinterpret_cast<const float2 *>(gst + rr * D + c0);
                         } else if constexpr (kGate == kGateBF16) {
                             const uint32_t w = gbf[rr * (D / 2) + cp];
-                            gr = make_float2(lo_bf(w), hi_bf(w));
+                            gv[i] = make_float2(lo_bf(w), hi_bf(w));
                         } else {
-                            gr = make_float2(gsc[rr], gsc[rr]);
+                            gv[i] = make_float2(gsc[rr], gsc[rr]);
                         }
-                        if (act) {
-                            // g holds the gate's pre-activation: log alpha = logsigmoid(g); rows past
-                            // the end of the sequence keep log alpha = 0
-                            gv[i] = rr < Lrows ? make_float2(log2_sigmoid(gr.x), log2_sigmoid(gr.y))
-                                               : make_float2(0.f, 0.f);
-                        } else {
-                            gv[i] = f2_mul(gr, l2e);
-                        }
-                        gv[i] = make_float2(fmaxf(gv[i].x, kFloorLog2), fmaxf(gv[i].y, kFloorLog2));
-                        sp[i >> 3] = f2_add(sp[i >> 3], gv[i]);
                     }
+                    if (act) {
+                        // g holds the gate's pre-activation: log alpha = logsigmoid(g); rows past the
+                        // end of the sequence keep log alpha = 0
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int rr = (i < 8 ? rp0 : rp1) + (i & 7);
+                            gv[i] = rr < Lrows ? make_float2(log2_sigmoid(gv[i].x), log2_sigmoid(gv[i].y))
+                                               : make_float2(0.f, 0.f);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) gv[i] = f2_mul(gv[i], l2e);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) sp[i >> 3] = f2_add(sp[i >> 3], gv[i]);
                     // row-quarter sums of g per channel, [4][128] floats in the solve's scratch
                     float *gq = reinterpret_cast<float *>(sgen + PR_P);
                     const float2 qsum = f2_add(sp[0], sp[1]);
@@ -1119,6 +1126,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (named_bar_any(2, 256, unsafe || *abort_flag != 0)) {
                         if (named_bar_any(2, 256, *abort_flag != 0)) break;
                         robust = true;
+                        // the sub-block path floors the gates: again with the floored sums
+                        sp[0] = sp[1] = make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            gv[i] = make_float2(fmaxf(gv[i].x, kFloorLog2), fmaxf(gv[i].y, kFloorLog2));
+                            sp[i >> 3] = f2_add(sp[i >> 3], gv[i]);
+                        }
+                        *reinterpret_cast<float2 *>(gq + tq * 128 + c0) = f2_add(sp[0], sp[1]);
+                        if (named_bar_any(2, 256, *abort_flag != 0)) break;
                     }
                     float2 qs[4];
 #pragma unroll
@@ -1739,7 +1755,7 @@ cudaError_t noalloc_scratch(int dev, unsigned char **out) {
 }
 
 // Encode the tensor maps and launch one 4-CTA cluster per (sequence, head).
-template <bool kRingPerCluster, int kGate, bool kNorm>
+template <bool kRingPerCluster, int kGate, bool kNorm, bool kSeg = false>
 cudaError_t launch_clusters(const FwdParams &p, int64_t rows, int64_t grid, unsigned char *rings,
                             cudaStream_t stream) {
     tc::TmaMaps maps;
@@ -1760,7 +1776,7 @@ cudaError_t launch_clusters(const FwdParams &p, int64_t rows, int64_t grid, unsi
                       CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
-    cudaError_t err = cudaFuncSetAttribute(tc::kda_fwd_tc_kernel<kRingPerCluster, kGate, kNorm>,
+    cudaError_t err = cudaFuncSetAttribute(tc::kda_fwd_tc_kernel<kRingPerCluster, kGate, kNorm, kSeg>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(tc::SMEM_BYTES));
     if (err != cudaSuccess) return err;
@@ -1776,7 +1792,7 @@ cudaError_t launch_clusters(const FwdParams &p, int64_t rows, int64_t grid, unsi
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, tc::kda_fwd_tc_kernel<kRingPerCluster, kGate, kNorm>, p, maps, rings);
+    err = cudaLaunchKernelEx(&cfg, tc::kda_fwd_tc_kernel<kRingPerCluster, kGate, kNorm, kSeg>, p, maps, rings);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
@@ -1794,6 +1810,11 @@ cudaError_t launch_fwd_tc(const FwdParams &p, int64_t rows, cudaStream_t stream)
     unsigned char *rings = ring_pool(dev);
     if (!rings) return cudaErrorMemoryAllocation;
     const bool norm = (p.flags & kFlagL2NormQK) != 0;
+    if (p.seg_len > 0 || p.mode != kModePlain) {
+        // the segmented forward takes the plain gate only
+        if (p.gate_mode != kGateF32 || p.flags != 0) return cudaErrorInvalidValue;
+        return launch_clusters<false, kGateF32, false, true>(p, rows, grid, rings, stream);
+    }
     switch (p.gate_mode) {
         case kGateF32:
             return norm ? launch_clusters<false, kGateF32, true>(p, rows, grid, rings, stream)
