@@ -195,6 +195,43 @@ kda_status kda_fwd_segmented(const void *q, const void *k, const void *v, const 
                              size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * kda_bwd -- gradients of the chunkwise forward: of L = sum(dout . out) +
+ * sum(dfinal_state . final_state) with respect to q, k, v, g, beta and the initial
+ * state.
+ *
+ * The FlashKDA release page describes the library as forward and backward kernels
+ * for KDA; this is the backward of kda_fwd's operator (the state-update equation of
+ * the Kimi Linear feature page, chapter 4), for training. It runs the chunk form of
+ * the recurrence backwards, last chunk first, in chunks of 16 tokens, in fp32: a
+ * forward sweep stores the state entering every 64 tokens in `workspace`, and the
+ * reverse sweep recomputes each chunk from its stored state.
+ *
+ * Inputs are kda_fwd's (q, k, v bf16, g fp32 log alpha per channel, beta fp32,
+ * cu_seqlens, initial_state bf16/fp32/NULL, same layouts and rules) plus:
+ *   dout           bf16 [batch, seq_len, num_heads, 128]: dL/d out
+ *   dfinal_state   fp32 [num_seqs_eff, num_heads, 128, 128] or NULL (zero): dL/d final state
+ * Outputs (fp32, written; every pointer 16-byte aligned, dbeta 4-byte):
+ *   dq, dk, dv, dg [batch, seq_len, num_heads, 128];  dbeta [batch, seq_len, num_heads]
+ *   dinitial_state [num_seqs_eff, num_heads, 128, 128], or NULL (not written)
+ *   workspace      caller-owned device memory, 256-byte aligned, at least
+ *                  kda_bwd_workspace(total_tokens, num_seqs_eff, num_heads) bytes
+ *                  (64 KiB per 64 tokens per head, plus one state per sequence
+ *                  and head); contents on entry do not matter.
+ * total_tokens is batch * seq_len (seq_len with cu_seqlens). The gates are taken
+ * as in kda_fwd's sub-block path: a per-token log-decay below -10 counts as -10,
+ * and its gradient is 0. dq, dk, dg and dbeta gather four partial sums by fp32
+ * atomic adds, so they can differ from run to run in the last bits.
+ * KDA_ERR_WORKSPACE if the workspace is smaller than needed.
+ */
+size_t kda_bwd_workspace(int64_t total_tokens, int32_t num_seqs, int32_t num_heads);
+kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta, float scale,
+                   const int32_t *cu_seqlens, int32_t num_seqs, int32_t batch, int64_t seq_len, int32_t num_heads,
+                   int32_t head_dim_k, int32_t head_dim_v, const void *initial_state, kda_dtype initial_dtype,
+                   const void *dout, const float *dfinal_state, float *dq, float *dk, float *dv, float *dg,
+                   float *dbeta, float *dinitial_state, void *workspace, size_t workspace_bytes,
+                   kda_stream_t stream);
+
+/*
  * kda_fwd_noalloc -- kda_fwd for callers that cannot allocate device memory.
  *
  * The method's pages define no such call; it exists for the library's own

@@ -16,8 +16,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libkda.so")
 
 # entry points declared in include/kda.h
-EXPORTS = ("kda_decode", "kda_device_error", "kda_fwd", "kda_fwd_ex", "kda_fwd_noalloc", "kda_fwd_segmented",
-           "kda_fwd_segmented_workspace", "kda_status_string", "kda_version")
+EXPORTS = ("kda_bwd", "kda_bwd_workspace", "kda_decode", "kda_device_error", "kda_fwd", "kda_fwd_ex",
+           "kda_fwd_noalloc", "kda_fwd_segmented", "kda_fwd_segmented_workspace", "kda_status_string",
+           "kda_version")
 
 # kda_fwd_ex gate kinds and flags (include/kda.h)
 KDA_GATE_FP32, KDA_GATE_BF16, KDA_GATE_SCALAR_FP32 = 0, 1, 2
@@ -65,6 +66,11 @@ def load_library(path: str | None = None):
                                           P, ctypes.c_int, P, i64, P, ctypes.c_size_t, P]
         lib.kda_fwd_segmented_workspace.restype = ctypes.c_size_t
         lib.kda_fwd_segmented_workspace.argtypes = [i32, i64, i32, i64]
+        lib.kda_bwd.restype = ctypes.c_int
+        lib.kda_bwd.argtypes = [P, P, P, P, P, ctypes.c_float, P, i32, i32, i64, i32, i32, i32, P, ctypes.c_int,
+                                P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        lib.kda_bwd_workspace.restype = ctypes.c_size_t
+        lib.kda_bwd_workspace.argtypes = [i64, i32, i32]
         lib.kda_decode.restype = ctypes.c_int
         lib.kda_decode.argtypes = [P, P, P, P, P, ctypes.c_float, i32, i32, i32, i32, P, P, ctypes.c_int, P, P]
         lib.kda_status_string.restype = ctypes.c_char_p
@@ -281,6 +287,68 @@ def kda_fwd_segmented(q, k, v, g, beta, segment_len: int, scale: float | None = 
     if st != 0:
         raise KdaError(st, lib.kda_status_string(st).decode())
     return out, final_state
+
+
+def kda_bwd(q, k, v, g, beta, dout, scale: float | None = None, cu_seqlens=None, initial_state=None,
+            dfinal_state=None, want_dinitial_state: bool = True, workspace=None, stream=None):
+    """Gradients of sum(dout * out) + sum(dfinal_state * final_state) of ``kda_fwd`` with
+    respect to q, k, v, g, beta and the initial state (see include/kda.h, kda_bwd).
+
+    Inputs as for ``kda_fwd`` (fp32 per-channel g), plus dout bf16 [B, T, H, 128] and
+    dfinal_state fp32 [N, H, 128, 128] or None. Returns a dict of fp32 tensors: dq, dk, dv,
+    dg [B, T, H, 128], dbeta [B, T, H] and dh0 [N, H, 128, 128] (None unless asked).
+    ``workspace`` (uint8, at least ``bwd_workspace_bytes(...)``) is allocated when not given."""
+    import torch
+    _check("q", q, torch.bfloat16, 4)
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1] if v.dim() == 4 else -1
+    _check("k", k, torch.bfloat16, shape=q.shape)
+    _check("v", v, torch.bfloat16, shape=(B, T, H, Dv))
+    _check("g", g, torch.float32, shape=q.shape)
+    _check("beta", beta, torch.float32, shape=(B, T, H))
+    _check("dout", dout, torch.bfloat16, shape=(B, T, H, Dv))
+    if cu_seqlens is not None:
+        _check("cu_seqlens", cu_seqlens, torch.int32, 1)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    state_shape = (N, H, Dk, Dv)
+    if initial_state is not None:
+        _check("initial_state", initial_state, None, shape=state_shape)
+    if dfinal_state is not None:
+        _check("dfinal_state", dfinal_state, torch.float32, shape=state_shape)
+    if workspace is not None:
+        _check("workspace", workspace, torch.uint8, 1)
+    dev = _check_devices(q=q, k=k, v=v, g=g, beta=beta, dout=dout, cu_seqlens=cu_seqlens,
+                         initial_state=initial_state, dfinal_state=dfinal_state, workspace=workspace)
+    lib = load_library()
+    rows = T if cu_seqlens is not None else B * T
+    if workspace is None:
+        workspace = torch.empty(max(1, int(lib.kda_bwd_workspace(int(rows), int(N), int(H)))),
+                                dtype=torch.uint8, device=dev)
+    out = {n: torch.empty((B, T, H, Dk if n != "dv" else Dv), dtype=torch.float32, device=dev)
+           for n in ("dq", "dk", "dv", "dg")}
+    out["dbeta"] = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    out["dh0"] = torch.empty(state_shape, dtype=torch.float32, device=dev) if want_dinitial_state else None
+    if scale is None:
+        scale = Dk ** -0.5
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    ic = _dtype_code(initial_state)
+    with torch.cuda.device(dev):
+        st = lib.kda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(cu_seqlens), int(N),
+                         int(B), int(T), int(H), int(Dk), int(Dv), _ptr(initial_state), ic if ic >= 0 else 99,
+                         _ptr(dout), _ptr(dfinal_state), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                         _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dh0"]), _ptr(workspace),
+                         int(workspace.numel()), ctypes.c_void_p(int(stream)))
+    if st != 0:
+        raise KdaError(st, lib.kda_status_string(st).decode())
+    return out
+
+
+def bwd_workspace_bytes(total_tokens: int, num_seqs: int, num_heads: int) -> int:
+    """Bytes of workspace kda_bwd needs."""
+    return int(load_library().kda_bwd_workspace(int(total_tokens), int(num_seqs), int(num_heads)))
 
 
 def segmented_workspace_bytes(batch: int, seq_len: int, num_heads: int, segment_len: int) -> int:

@@ -215,6 +215,73 @@ kda_status kda_fwd_segmented(const void *q, const void *k, const void *v, const 
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+size_t kda_bwd_workspace(int64_t total_tokens, int32_t num_seqs, int32_t num_heads) {
+    if (total_tokens < 0 || num_seqs < 0 || num_heads < 1) return 0;
+    return kda::bwd_workspace_bytes(total_tokens, num_seqs, num_heads);
+}
+
+kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta, float scale,
+                   const int32_t *cu_seqlens, int32_t num_seqs, int32_t batch, int64_t seq_len, int32_t num_heads,
+                   int32_t head_dim_k, int32_t head_dim_v, const void *initial_state, kda_dtype initial_dtype,
+                   const void *dout, const float *dfinal_state, float *dq, float *dk, float *dv, float *dg,
+                   float *dbeta, float *dinitial_state, void *workspace, size_t workspace_bytes,
+                   kda_stream_t stream) {
+    // the forward's argument rules (no final state here; dinitial_state takes its place)
+    kda::FwdParams fp;
+    int64_t rows = 0;
+    kda_status st = prepare(q, k, v, g, beta, scale, cu_seqlens, num_seqs, batch, seq_len, num_heads, head_dim_k,
+                            head_dim_v, initial_state, initial_dtype, nullptr, KDA_DTYPE_NONE, dq, false,
+                            KDA_GATE_FP32, 0u, &fp, &rows);
+    if (st != KDA_OK) return st;
+    if (rows > 0 && (!dout || !dk || !dv || !dg || !dbeta)) return KDA_ERR_NULL_PTR;
+    if (!aligned16(dout) || !aligned16(dk) || !aligned16(dv) || !aligned16(dg) || !aligned16(dfinal_state) ||
+        !aligned16(dinitial_state) || (reinterpret_cast<uintptr_t>(dbeta) & 3u))
+        return KDA_ERR_BAD_ALIGNMENT;
+    if (fp.num_seqs == 0) return KDA_OK;
+    const size_t need = kda::bwd_workspace_bytes(rows, fp.num_seqs, num_heads);
+    if (!workspace) return KDA_ERR_NULL_PTR;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KDA_ERR_BAD_ALIGNMENT;
+    if (workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // dq, dk, dg and dbeta gather the value-column slices' shares; dv too is cleared, for tokens
+    // that no sequence covers
+    const size_t elems = static_cast<size_t>(rows) * num_heads * kda::kHeadDim;
+    cudaError_t err = cudaSuccess;
+    if (rows > 0) {
+        if (err == cudaSuccess) err = cudaMemsetAsync(dq, 0, elems * sizeof(float), s);
+        if (err == cudaSuccess) err = cudaMemsetAsync(dk, 0, elems * sizeof(float), s);
+        if (err == cudaSuccess) err = cudaMemsetAsync(dv, 0, elems * sizeof(float), s);
+        if (err == cudaSuccess) err = cudaMemsetAsync(dg, 0, elems * sizeof(float), s);
+        if (err == cudaSuccess)
+            err = cudaMemsetAsync(dbeta, 0, static_cast<size_t>(rows) * num_heads * sizeof(float), s);
+    }
+    if (err != cudaSuccess) return KDA_ERR_CUDA;
+    kda::BwdParams p;
+    p.q = fp.q;
+    p.k = fp.k;
+    p.v = fp.v;
+    p.g = static_cast<const float *>(fp.g);
+    p.beta = fp.beta;
+    p.scale = scale;
+    p.cu_seqlens = cu_seqlens;
+    p.seq_len = seq_len;
+    p.num_seqs = fp.num_seqs;
+    p.num_heads = num_heads;
+    p.h0 = initial_state;
+    p.h0_fp32 = initial_dtype == KDA_DTYPE_FP32;
+    p.dout = static_cast<const uint16_t *>(dout);
+    p.dhT = dfinal_state;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.dg = dg;
+    p.dbeta = dbeta;
+    p.dh0 = dinitial_state;
+    p.workspace = static_cast<float *>(workspace);
+    err = kda::launch_bwd(p, s);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status kda_fwd_noalloc(const void *q, const void *k, const void *v, const float *g,
                            const float *beta, float scale, const int32_t *cu_seqlens,
                            int32_t num_seqs, int32_t batch, int64_t seq_len, int32_t num_heads,

@@ -64,6 +64,27 @@ cudaError_t launch_fwd_tc_noalloc(const FwdParams &p, int64_t rows, cudaStream_t
 cudaError_t launch_segment_scan(const void *h0, int h0_fp32, const float *M, const float *B, float *S_in,
                                 int32_t rows, int32_t seg_count, int32_t num_heads, cudaStream_t stream);
 
+// Backward pass (kda_bwd.cu): gradients of sum(dout . out) + sum(dhT . hT).
+struct BwdParams {
+    const uint16_t *q, *k, *v;  // bf16 bits, [rows, H, 128]
+    const float *g;             // [rows, H, 128], log alpha
+    const float *beta;          // [rows, H]
+    float scale;
+    const int32_t *cu_seqlens;  // device, or nullptr (fixed-length rows)
+    int64_t seq_len;
+    int32_t num_seqs;
+    int32_t num_heads;
+    const void *h0;             // [num_seqs, H, 128, 128] or nullptr
+    int32_t h0_fp32;
+    const uint16_t *dout;       // bf16 [rows, H, 128]
+    const float *dhT;           // [num_seqs, H, 128, 128] or nullptr
+    float *dq, *dk, *dv, *dg, *dbeta;  // zeroed by the caller's launch sequence (dq, dk, dg, dbeta)
+    float *dh0;                 // [num_seqs, H, 128, 128] or nullptr
+    float *workspace;           // checkpoint states, bwd_workspace_bytes
+};
+size_t bwd_workspace_bytes(int64_t rows, int64_t num_seqs, int32_t num_heads);
+cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream);
+
 // Bits of the device-side error word shared by the library's kernels.
 constexpr unsigned int kErrTimeout = 1u;    // a bounded wait gave up; the kernel wound down early
 constexpr unsigned int kErrRingIndex = 2u;  // a chain CTA ran on an SM id beyond the ring pool

@@ -186,3 +186,11 @@ def test_segmented_workspace_size(lib):
     assert f(1, 1 << 20, 32, 1 << 15) == 3 * 32 * 32 * 128 * 128 * 4
     assert f(2, 1000, 3, 192) == 3 * 2 * 6 * 3 * 128 * 128 * 4
     assert f(1, 1000, 3, 100) == 0 and f(1, 1000, 3, 0) == 0 and f(1, 1000, 0, 64) == 0
+
+
+def test_bwd_workspace_size(lib):
+    f = lib.kda_bwd_workspace
+    # one 128 x 128 fp32 state per 64 tokens per head, plus one per sequence and head, plus one
+    assert f(4096, 1, 32) == (64 + 1 + 1) * 32 * 65536
+    assert f(1000, 3, 2) == (15 + 3 + 1) * 2 * 65536
+    assert f(-1, 1, 1) == 0 and f(10, 1, 0) == 0
