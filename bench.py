@@ -54,6 +54,27 @@ def decode_unit_bytes(state_dtype: str) -> int:
     return 2 * D * D * esz + 4 * D * 2 + D * 4 + 4
 
 
+def bwd_flops_per_token_head(C: int = 16) -> float:
+    """FLOPs per token and head of the backward's chunk algebra (kda_bwd, chunks of C
+    tokens), each dense product counted once (the kernel's recomputation not counted):
+    X, S, dQd, dKt, dD (state part), dKd and dS's two products at C x D x D each; dGl and
+    the decay of dS at D x D; B, Aqk, dAqk and the four decayed products of dK and dQ at
+    C (C + 1) / 2 x D; D, dD (intra part), dTp, dX at C x C x D; dAkk at 2 C^3."""
+    fma = (8 * C * D * D + 2 * D * D + 7 * (C * (C + 1) // 2) * D + 4 * C * C * D + 2 * C ** 3)
+    return 2.0 * fma / C
+
+
+# algorithmic HBM bytes per token and head of the backward: q, k, v, dout read (bf16),
+# g (fp32) and beta read; dq, dk, dv, dg (fp32) and dbeta written; the 64 KiB state
+# checkpoint per 64 tokens written once and read once
+BWD_BYTES_PER_TOKEN_HEAD = 4 * 2 * D + 4 * D + 4 + 4 * 4 * D + 4 + 2 * (4 * D * D) // 64
+
+
+def fp32_alu_peak_tflops(sm_max_mhz: float, sms: int = 148) -> float:
+    """fp32 FMA peak of the CUDA cores: 128 lanes per SM, 2 FLOP per FMA, at the SM clock."""
+    return sms * 128 * 2 * sm_max_mhz * 1e6 / 1e12
+
+
 def state_bytes(N, H, init_dt, final_dt) -> int:
     b = 0
     for dt in (init_dt, final_dt):
@@ -216,6 +237,8 @@ def cpu_baseline_run(inp, tokens_per_step, steps=1, warmup=0):
     sample = {}
     for name in ("q", "k", "v", "g", "beta"):
         sample[name] = inp[name][:1, :tokens_per_step].cpu().float().contiguous()
+    if sample["g"].dim() == 3:   # one decay per token and head: the same on every channel
+        sample["g"] = sample["g"][..., None].expand(*sample["g"].shape, D).contiguous()
     h0 = None if inp["h0"] is None else inp["h0"][:1].cpu().double()
     threads = os.cpu_count() or 1
     times = []
@@ -323,6 +346,13 @@ def main():
     ap.add_argument("--split", default="none", choices=["none", "heads"],
                     help="none: each rank runs its own copy of the workload (weak scaling); "
                          "heads: the ranks share the workload's heads (strong scaling)")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward pass (kda_bwd) on the workload instead; prints its own line")
+    ap.add_argument("--segmented", type=int, default=0, metavar="TOKENS",
+                    help="time kda_fwd_segmented with pieces of TOKENS tokens instead of kda_fwd")
+    ap.add_argument("--heads", type=int, default=0, help="override the workload's number of heads")
+    ap.add_argument("--gate", default="fp32", choices=["fp32", "bf16", "per_token"],
+                    help="gate input of the timed forward (kda_fwd_ex for bf16 and per_token)")
     ap.add_argument("--decode", default=None, metavar="BxH[:bf16]",
                     help="time the single-token decode step instead (e.g. 256x32 or 256x32:bf16); "
                          "prints its own line, not the prefill metric")
@@ -330,6 +360,8 @@ def main():
     args.warmup = max(args.warmup, 3)
     if args.decode:
         return decode_main(args)
+    if args.bwd:
+        return bwd_main(args)
 
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         return relaunch_under_torchrun(args.gpus)
@@ -360,18 +392,33 @@ def main():
         del full
         torch.cuda.empty_cache()
     else:
-        inp = make_inputs(name, device="cuda", seed=rank_seed(cfg["seed"], rank))
+        over = {"H": args.heads} if args.heads else {}
+        inp = make_inputs(name, device="cuda", seed=rank_seed(cfg["seed"], rank), **over)
         H_all = inp["H"]
+    if args.gate == "bf16":
+        inp["g"] = inp["g"].to(torch.bfloat16)
+    elif args.gate == "per_token":
+        inp["g"] = inp["g"][..., 0].contiguous()
     H, N, tokens = inp["H"], inp["N"], inp["B"] * inp["T"]
     final_dt = inp["final_dtype"]
     out = torch.empty_like(inp["v"])
     hT = None if final_dt is None else torch.empty((N, H, D, D), dtype=final_dt, device="cuda")
     stream = torch.cuda.current_stream()
 
+    seg_ws = None
+    if args.segmented:
+        seg_ws = torch.empty(max(1, kda.segmented_workspace_bytes(inp["B"], inp["T"], H, args.segmented)),
+                             dtype=torch.uint8, device="cuda")
+
     def step():
-        kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["scale"],
-                    cu_seqlens=inp["cu_seqlens"], initial_state=inp["h0"], final_state=hT,
-                    out=out)
+        if args.segmented:
+            kda.kda_fwd_segmented(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], args.segmented,
+                                  inp["scale"], initial_state=inp["h0"], final_state=hT, out=out,
+                                  workspace=seg_ws)
+        else:
+            kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["scale"],
+                        cu_seqlens=inp["cu_seqlens"], initial_state=inp["h0"], final_state=hT,
+                        out=out)
 
     for _ in range(args.warmup):
         step()
@@ -404,15 +451,22 @@ def main():
     value = (tokens / (ms_per_step / 1e3)) if strong else whole_job_value(world, tokens, ms_per_step)
     flops = pages_flops(tokens, H_all) if strong else world * pages_flops(tokens, H)
     peaks = load_peaks()
-    alg_bytes = tokens * H * BYTES_PER_TOKEN_HEAD + state_bytes(
+    # a bf16 gate saves 256 B per token-head, a per-token one 508 B
+    bytes_th = BYTES_PER_TOKEN_HEAD - {"fp32": 0, "bf16": 2 * D, "per_token": 4 * D - 4}[args.gate]
+    alg_bytes = tokens * H * bytes_th + state_bytes(
         N, H, None if inp["h0"] is None else inp["h0"].dtype, final_dt)
     avg_launch_s = statistics.mean(launch_ms) / 1e3
     achieved_gbs = alg_bytes / avg_launch_s / 1e9
     traffic, prof_kernel = profiled_traffic(tokens * H)
+    if args.segmented or args.gate != "fp32":
+        # the committed DRAM counters are the plain kernel's
+        traffic = None
+        prof_kernel = ("kda_fwd_segmented (affine run, scan, forward run)" if args.segmented
+                       else f"kda_fwd_ex ({args.gate} gate)")
 
     # ---- end to end: pinned host buffers -> device -> kda_fwd -> host, per step
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.gate == "fp32" and not args.segmented:
         e2e = e2e_run(args, inp, world, rank, strong=strong)
 
     cpu = None
@@ -440,7 +494,8 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "strong" if strong else "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(name, world, split=args.split),
+            "config": dict(workload_config(name, world, split=args.split), heads=H_all, gate=args.gate,
+                           **({"segment_len": args.segmented} if args.segmented else {})),
             "tflops": flops / (ms_per_step / 1e3) / 1e12,
             "frac_bf16_peak": flops / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"] / world,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
@@ -450,7 +505,7 @@ def main():
                          "alg_bytes_per_launch": alg_bytes,
                          "avg_launch_ms": avg_launch_s * 1e3},
             "cpu_baseline": cpu, "e2e": e2e, "parity": parity,
-            "gpu_launches": args.steps * 1,
+            "gpu_launches": args.steps * (3 if args.segmented else 1),
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -468,6 +523,65 @@ def current_gpu_sampler():
     uuid = str(getattr(props, "uuid", ""))
     return ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else
                         (uuid or torch.cuda.current_device()))
+
+
+def bwd_main(args):
+    """The backward pass (kda_bwd) on one GPU over the workload (default: the 4K-token one),
+    with seeded bf16 output gradients and an fp32 final-state gradient."""
+    import torch
+    import kimi_delta_attention_27_b200 as kda
+    from kimi_delta_attention_27_b200.inputs import make_inputs
+    name = args.workload if args.workload != "t1m_h32" else "t4k_h32"
+    over = {"H": args.heads} if args.heads else {}
+    inp = make_inputs(name, device="cuda", **over)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(77)
+    dout = torch.randn(inp["v"].shape, generator=gen, device="cuda").to(torch.bfloat16)
+    dhT = torch.randn((inp["N"], inp["H"], D, D), generator=gen, device="cuda")
+    H, tokens = inp["H"], inp["B"] * inp["T"]
+    ws = torch.empty(kda.bwd_workspace_bytes(tokens, inp["N"], H), dtype=torch.uint8, device="cuda")
+
+    def step():
+        return kda.kda_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], dout, inp["scale"],
+                           cu_seqlens=inp["cu_seqlens"], initial_state=inp["h0"], dfinal_state=dhT, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = current_gpu_sampler()
+    sampler.start()
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream()
+    t0 = torch.cuda.Event(enable_timing=True); t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    peaks = load_peaks()
+    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else io.StringIO("{}") as f:
+        sm_max = float(json.load(f).get("sm_max_mhz", 1965.0))
+    flops = tokens * H * bwd_flops_per_token_head()
+    achieved = flops / (ms / 1e3) / 1e12
+    peak = fp32_alu_peak_tflops(sm_max)
+    line = {
+        "metric": "KDA bwd tokens/s (dq, dk, dv, dg, dbeta, dh0)", "value": tokens / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(name, 1), heads=H),
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "kda::bwd::kda_bwd_kernel",
+                     "flops_per_token_head": bwd_flops_per_token_head(),
+                     "peak_source": f"derived: 148 SMs x 128 fp32 lanes x 2 x {sm_max:.0f} MHz",
+                     "hbm_bytes_per_token_head": BWD_BYTES_PER_TOKEN_HEAD,
+                     "hbm_gbs": tokens * H * BWD_BYTES_PER_TOKEN_HEAD / (ms / 1e3) / 1e9,
+                     "hbm_peak_gbs": peaks["hbm_gbs"]},
+        "gpu_launches": args.steps * 1, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
 
 
 def decode_main(args):

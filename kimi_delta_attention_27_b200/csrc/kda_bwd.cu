@@ -52,6 +52,7 @@ constexpr int VS = D / NV;       // 32 value columns per CTA
 constexpr int VP = VS + 1;       // padded row pitch of a state slice: rows c, c + 1 in distinct banks
 constexpr int NT = 256;
 constexpr int AP = CB + 1;       // pitch of the CB x CB matrices
+constexpr int DP = D + 1;        // pitch of the CB x D tiles: 16 lanes reading one column of 16 rows hit distinct banks
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kFloorLog2 = -14.426950408889634f;   // log2 of e^-10
 
@@ -59,18 +60,18 @@ constexpr float kFloorLog2 = -14.426950408889634f;   // log2 of e^-10
 constexpr int SM_SCK = 0;                          // NSUB states [D][VP] entering the group's chunks
 constexpr int SM_DS = SM_SCK + NSUB * D * VP;      // dS [D][VP]
 constexpr int SM_K = SM_DS + D * VP;               // [CB][D] each: K, Q, G (log2 units)
-constexpr int SM_Q = SM_K + CB * D;
-constexpr int SM_G = SM_Q + CB * D;
-constexpr int SM_KD = SM_G + CB * D;               // Kd, Qd, Kt
-constexpr int SM_QD = SM_KD + CB * D;
-constexpr int SM_KT = SM_QD + CB * D;
-constexpr int SM_KL = SM_KT + CB * D;              // K e^(G - Ga), Q e^(G - Ga), K e^(Ga - G)
-constexpr int SM_QL = SM_KL + CB * D;
-constexpr int SM_KR = SM_QL + CB * D;
-constexpr int SM_P1 = SM_KR + CB * D;              // partial sums [CB][D]: dQd, dKt, dKd
-constexpr int SM_P2 = SM_P1 + CB * D;
-constexpr int SM_P3 = SM_P2 + CB * D;
-constexpr int SM_V = SM_P3 + CB * D;               // [CB][VP] slices: V, dO, X, D, dD, dX
+constexpr int SM_Q = SM_K + CB * DP;
+constexpr int SM_G = SM_Q + CB * DP;
+constexpr int SM_KD = SM_G + CB * DP;              // Kd, Qd, Kt
+constexpr int SM_QD = SM_KD + CB * DP;
+constexpr int SM_KT = SM_QD + CB * DP;
+constexpr int SM_KL = SM_KT + CB * DP;             // K e^(G - Ga), Q e^(G - Ga), K e^(Ga - G)
+constexpr int SM_QL = SM_KL + CB * DP;
+constexpr int SM_KR = SM_QL + CB * DP;
+constexpr int SM_P1 = SM_KR + CB * DP;             // partial sums [CB][D]: dQd, dKt, dKd
+constexpr int SM_P2 = SM_P1 + CB * DP;
+constexpr int SM_P3 = SM_P2 + CB * DP;
+constexpr int SM_V = SM_P3 + CB * DP;              // [CB][VP] slices: V, dO, X, D, dD, dX
 constexpr int SM_DO = SM_V + CB * VP;
 constexpr int SM_X = SM_DO + CB * VP;
 constexpr int SM_DD = SM_X + CB * VP;
@@ -137,13 +138,13 @@ __device__ void load_chunk(const BwdParams &p, const Unit &u, int64_t t0, int L,
         if (r < L) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                sm[SM_K + r * D + c0 + e] = bf(p.k[off + e]);
-                sm[SM_Q + r * D + c0 + e] = bf(p.q[off + e]);
-                sm[SM_G + r * D + c0 + e] = fmaxf(p.g[off + e] * kLog2e, kFloorLog2);
+                sm[SM_K + r * DP + c0 + e] = bf(p.k[off + e]);
+                sm[SM_Q + r * DP + c0 + e] = bf(p.q[off + e]);
+                sm[SM_G + r * DP + c0 + e] = fmaxf(p.g[off + e] * kLog2e, kFloorLog2);
             }
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) sm[SM_K + r * D + c0 + e] = sm[SM_Q + r * D + c0 + e] = sm[SM_G + r * D + c0 + e] = 0.f;
+            for (int e = 0; e < 8; ++e) sm[SM_K + r * DP + c0 + e] = sm[SM_Q + r * DP + c0 + e] = sm[SM_G + r * DP + c0 + e] = 0.f;
         }
     }
     {   // V and dO slices: thread t takes row t >> 4, columns 2 (t & 15) .. + 2 of the slice
@@ -170,8 +171,8 @@ __device__ void load_chunk(const BwdParams &p, const Unit &u, int64_t t0, int L,
         float run = 0.f;
 #pragma unroll
         for (int r = 0; r < CB; ++r) {
-            run += sm[SM_G + r * D + t];
-            sm[SM_G + r * D + t] = run;
+            run += sm[SM_G + r * DP + t];
+            sm[SM_G + r * DP + t] = run;
         }
         sm[SM_EC + t] = ex2(run);
     }
@@ -182,15 +183,15 @@ __device__ void load_chunk(const BwdParams &p, const Unit &u, int64_t t0, int L,
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const int c = (t & 15) + 16 * e;
-            const float gr = sm[SM_G + r * D + c], ga = sm[SM_G + 7 * D + c], gl = sm[SM_G + (CB - 1) * D + c];
-            const float k = sm[SM_K + r * D + c], q = sm[SM_Q + r * D + c];
+            const float gr = sm[SM_G + r * DP + c], ga = sm[SM_G + 7 * DP + c], gl = sm[SM_G + (CB - 1) * DP + c];
+            const float k = sm[SM_K + r * DP + c], q = sm[SM_Q + r * DP + c];
             const float ed = ex2(gr), el = ex2(gr - ga), er = ex2(ga - gr);
-            sm[SM_KD + r * D + c] = k * ed;
-            sm[SM_QD + r * D + c] = q * ed;
-            sm[SM_KT + r * D + c] = k * ex2(gl - gr);
-            sm[SM_KL + r * D + c] = k * el;
-            sm[SM_QL + r * D + c] = q * el;
-            sm[SM_KR + r * D + c] = k * er;
+            sm[SM_KD + r * DP + c] = k * ed;
+            sm[SM_QD + r * DP + c] = q * ed;
+            sm[SM_KT + r * DP + c] = k * ex2(gl - gr);
+            sm[SM_KL + r * DP + c] = k * el;
+            sm[SM_QL + r * DP + c] = q * el;
+            sm[SM_KR + r * DP + c] = k * er;
         }
     }
     __syncthreads();
@@ -205,9 +206,9 @@ __device__ void chunk_blocks(float *sm) {
         if (i <= r) {
 #pragma unroll 8
             for (int c = 0; c < D; ++c) {
-                const float kr = sm[SM_KR + i * D + c];
-                b = fmaf(sm[SM_KL + r * D + c], kr, b);
-                a = fmaf(sm[SM_QL + r * D + c], kr, a);
+                const float kr = sm[SM_KR + i * DP + c];
+                b = fmaf(sm[SM_KL + r * DP + c], kr, b);
+                a = fmaf(sm[SM_QL + r * DP + c], kr, a);
             }
         }
         sm[SM_B + r * AP + i] = b;
@@ -240,7 +241,7 @@ __device__ void chunk_xd(float *sm, const float *S0) {
         float x0 = sm[SM_V + r * VP + j0], x1 = sm[SM_V + r * VP + j0 + 1];
 #pragma unroll 8
         for (int c = 0; c < D; ++c) {
-            const float kd = sm[SM_KD + r * D + c];
+            const float kd = sm[SM_KD + r * DP + c];
             x0 = fmaf(-kd, S0[c * VP + j0], x0);
             x1 = fmaf(-kd, S0[c * VP + j0 + 1], x1);
         }
@@ -272,7 +273,7 @@ __device__ void chunk_state(float *sm, const float *S0, float *S1) {
     for (int e = 0; e < 16; ++e) acc[e] = ec * S0[c * VP + j0 + e];
 #pragma unroll
     for (int r = 0; r < CB; ++r) {
-        const float kt = sm[SM_KT + r * D + c];
+        const float kt = sm[SM_KT + r * DP + c];
 #pragma unroll
         for (int e = 0; e < 16; ++e) acc[e] = fmaf(kt, sm[SM_D + r * VP + j0 + e], acc[e]);
     }
@@ -389,8 +390,8 @@ __global__ void __launch_bounds__(NT, 1) kda_bwd_kernel(const BwdParams p) {
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    sm[SM_P1 + r * D + c0 + 16 * e] = scale * q8[e];
-                    sm[SM_P2 + r * D + c0 + 16 * e] = k8[e];
+                    sm[SM_P1 + r * DP + c0 + 16 * e] = scale * q8[e];
+                    sm[SM_P2 + r * DP + c0 + 16 * e] = k8[e];
                 }
             }
             {
@@ -425,7 +426,7 @@ __global__ void __launch_bounds__(NT, 1) kda_bwd_kernel(const BwdParams p) {
                 d1 *= scale;
 #pragma unroll 8
                 for (int c = 0; c < D; ++c) {
-                    const float kt = sm[SM_KT + r * D + c];
+                    const float kt = sm[SM_KT + r * DP + c];
                     d0 = fmaf(kt, dS[c * VP + j0], d0);
                     d1 = fmaf(kt, dS[c * VP + j0 + 1], d1);
                 }
@@ -470,7 +471,7 @@ __global__ void __launch_bounds__(NT, 1) kda_bwd_kernel(const BwdParams p) {
                     for (int e = 0; e < 8; ++e) a8[e] = fmaf(dx, S0[(c0 + 16 * e) * VP + j], a8[e]);
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) sm[SM_P3 + r * D + c0 + 16 * e] = -a8[e];
+                for (int e = 0; e < 8; ++e) sm[SM_P3 + r * DP + c0 + 16 * e] = -a8[e];
             }
             {
                 // dS <- scale Qd^T dO + Diag(e^Gl) dS - Kd^T dX (slice); each thread its own entries
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(NT, 1) kda_bwd_kernel(const BwdParams p) {
                 for (int e = 0; e < 16; ++e) acc[e] = ec * dS[c * VP + j0 + e];
 #pragma unroll
                 for (int r = 0; r < CB; ++r) {
-                    const float qd = scale * sm[SM_QD + r * D + c], kd = sm[SM_KD + r * D + c];
+                    const float qd = scale * sm[SM_QD + r * DP + c], kd = sm[SM_KD + r * DP + c];
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         acc[e] = fmaf(qd, sm[SM_DO + r * VP + j0 + e], fmaf(-kd, sm[SM_DX + r * VP + j0 + e], acc[e]));
@@ -528,12 +529,12 @@ __global__ void __launch_bounds__(NT, 1) kda_bwd_kernel(const BwdParams p) {
 #pragma unroll 2
                 for (int e = 0; e < 8; ++e) {
                     const int c = (t & 15) + 16 * e;
-                    const float gr = sm[SM_G + r * D + c], ga = sm[SM_G + 7 * D + c], gl = sm[SM_G + (CB - 1) * D + c];
+                    const float gr = sm[SM_G + r * DP + c], ga = sm[SM_G + 7 * DP + c], gl = sm[SM_G + (CB - 1) * DP + c];
                     const float lk = ex2(gr - ga), rs = ex2(ga - gr), ed = ex2(gr), et = ex2(gl - gr);
                     // (dB Kn) e^G and (dAqk Kn) e^G: lk * sum_i x[r][i] Kr[i]; dB = Diag(beta) dAkk
                     float bk = 0.f, ak = 0.f;
                     for (int i = 0; i <= r; ++i) {
-                        const float kr = sm[SM_KR + i * D + c];
+                        const float kr = sm[SM_KR + i * DP + c];
                         bk = fmaf(sm[SM_DAKK + r * AP + i], kr, bk);
                         ak = fmaf(sm[SM_DAQK + r * AP + i], kr, ak);
                     }
@@ -542,19 +543,19 @@ __global__ void __launch_bounds__(NT, 1) kda_bwd_kernel(const BwdParams p) {
                     // (dB^T Kd) e^-G and (dAqk^T Qd) e^-G: rs * sum_m x[m][r] Kl[m], Ql[m]
                     float bt = 0.f, at = 0.f;
                     for (int mm = r; mm < CB; ++mm) {
-                        bt = fmaf(sm[SM_DAKK + mm * AP + r] * sm[SM_BETA + mm], sm[SM_KL + mm * D + c], bt);
-                        at = fmaf(sm[SM_DAQK + mm * AP + r], sm[SM_QL + mm * D + c], at);
+                        bt = fmaf(sm[SM_DAKK + mm * AP + r] * sm[SM_BETA + mm], sm[SM_KL + mm * DP + c], bt);
+                        at = fmaf(sm[SM_DAQK + mm * AP + r], sm[SM_QL + mm * DP + c], at);
                     }
                     const float dkn = rs * (bt + at);                 // dKn e^-G
-                    const float dkd = sm[SM_P3 + r * D + c] * ed + bk;  // dKd e^G
-                    const float dqd = sm[SM_P1 + r * D + c] * ed + ak;  // dQd e^G = dQ
-                    const float dkt = sm[SM_P2 + r * D + c] * et;       // dKt e^(Gl - G)
-                    const float k = sm[SM_K + r * D + c], q = sm[SM_Q + r * D + c];
+                    const float dkd = sm[SM_P3 + r * DP + c] * ed + bk;  // dKd e^G
+                    const float dqd = sm[SM_P1 + r * DP + c] * ed + ak;  // dQd e^G = dQ
+                    const float dkt = sm[SM_P2 + r * DP + c] * et;       // dKt e^(Gl - G)
+                    const float k = sm[SM_K + r * DP + c], q = sm[SM_Q + r * DP + c];
                     float dgam = k * dkd + q * dqd - k * dkn - k * dkt;
-                    sm[SM_P1 + r * D + c] = dqd;
-                    sm[SM_P3 + r * D + c] = dkd + dkn + dkt;
-                    sm[SM_P2 + r * D + c] = k * dkt;   // dKt (.) Kt, summed over rows below
-                    sm[SM_KD + r * D + c] = dgam;      // Kd is not read again in this chunk
+                    sm[SM_P1 + r * DP + c] = dqd;
+                    sm[SM_P3 + r * DP + c] = dkd + dkn + dkt;
+                    sm[SM_P2 + r * DP + c] = k * dkt;   // dKt (.) Kt, summed over rows below
+                    sm[SM_KD + r * DP + c] = dgam;      // Kd is not read again in this chunk
                 }
             }
             __syncthreads();
@@ -563,12 +564,12 @@ __global__ void __launch_bounds__(NT, 1) kda_bwd_kernel(const BwdParams p) {
                 const int c = t;
                 float extra = sm[SM_DGL + c];
 #pragma unroll
-                for (int r = 0; r < CB; ++r) extra += sm[SM_P2 + r * D + c];
-                sm[SM_KD + (CB - 1) * D + c] += extra;
+                for (int r = 0; r < CB; ++r) extra += sm[SM_P2 + r * DP + c];
+                sm[SM_KD + (CB - 1) * DP + c] += extra;
                 float run = 0.f;
                 for (int r = CB - 1; r >= 0; --r) {
-                    run += sm[SM_KD + r * D + c];
-                    sm[SM_KD + r * D + c] = run;
+                    run += sm[SM_KD + r * DP + c];
+                    sm[SM_KD + r * DP + c] = run;
                 }
             }
             __syncthreads();
@@ -581,10 +582,10 @@ __global__ void __launch_bounds__(NT, 1) kda_bwd_kernel(const BwdParams p) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int c = (t & 15) + 16 * e;
-                        atomicAdd(&p.dq[off + c], sm[SM_P1 + r * D + c]);
-                        atomicAdd(&p.dk[off + c], sm[SM_P3 + r * D + c]);
+                        atomicAdd(&p.dq[off + c], sm[SM_P1 + r * DP + c]);
+                        atomicAdd(&p.dk[off + c], sm[SM_P3 + r * DP + c]);
                         // a log-decay raised to the floor has no gradient
-                        const float dg = p.g[off + c] * kLog2e >= kFloorLog2 ? sm[SM_KD + r * D + c] : 0.f;
+                        const float dg = p.g[off + c] * kLog2e >= kFloorLog2 ? sm[SM_KD + r * DP + c] : 0.f;
                         atomicAdd(&p.dg[off + c], dg);
                     }
                 }

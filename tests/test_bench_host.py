@@ -26,3 +26,18 @@ def test_decode_unit_bytes():
     # the state read and written, plus q, k, v, out (4 x 256 B), g (512 B) and beta (4 B)
     assert bench.decode_unit_bytes("fp32") == 2 * 65536 + 1540 == 132612
     assert bench.decode_unit_bytes("bf16") == 2 * 32768 + 1540 == 67076
+
+
+def test_backward_flop_and_byte_counts():
+    # C = 16, D = 128: eight C x D x D products, two D x D, seven triangular C (C + 1) / 2 x D,
+    # four C x C x D and 2 C^3, per chunk of 16 tokens, two FLOPs per multiply-add
+    C, D = 16, 128
+    per_chunk = 8 * C * D * D + 2 * D * D + 7 * (C * (C + 1) // 2) * D + 4 * C * C * D + 2 * C ** 3
+    assert per_chunk == 2391040
+    assert bench.bwd_flops_per_token_head() == 2 * per_chunk / C == 298880.0
+    # q, k, v, dout in; g, beta in; dq, dk, dv, dg, dbeta out; a 64 KiB checkpoint per 64 tokens, twice
+    assert bench.BWD_BYTES_PER_TOKEN_HEAD == 4 * 256 + 512 + 4 + 4 * 512 + 4 + 2 * 1024 == 5640
+
+
+def test_fp32_alu_peak():
+    assert abs(bench.fp32_alu_peak_tflops(1965.0) - 74.45) < 0.01
