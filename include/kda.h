@@ -101,13 +101,13 @@ typedef enum { KDA_DTYPE_NONE = 0, KDA_DTYPE_BF16 = 1, KDA_DTYPE_FP32 = 2 } kda_
  * scale multiplies the output (o_t = scale * S_t^T q_t); callers normally
  * pass 1/sqrt(128).
  *
- * Gate range: g may be any value <= 0, including -inf (alpha = 0). The kernel
- * raises per-token log-decays below -10 to -10 (alpha >= e^-10 = 4.5e-5): a
- * channel that keeps less than that of its state per token has forgotten it
- * to below the precision of its bf16 operands either way, and the change in
- * any output is bounded by e^-10 relative to the state it reads. Chunks whose
- * decay over either half exceeds 2^-100 on some channel take a slower path
- * with one decay anchor per 16 tokens instead of one per chunk.
+ * Gate range: g may be any value <= 0, including -inf (alpha = 0). A chunk in
+ * which some channel decays by more than 2^-50 over a 16-token quarter takes a
+ * slower path with one decay anchor per 16 tokens instead of one per chunk, and
+ * on that path per-token log-decays below -10 count as -10 (alpha >= e^-10 =
+ * 4.5e-5): a channel that keeps less than that of its state per token has
+ * forgotten it to below the precision of its bf16 operands either way, and the
+ * change in any state entry is at most e^-10 of the entry it decays.
  *
  * head_dim_k and head_dim_v must both be 128. All tensor pointers must be
  * 16-byte aligned (cu_seqlens 4-byte). Returns KDA_OK once the work is

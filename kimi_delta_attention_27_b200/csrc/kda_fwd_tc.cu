@@ -16,6 +16,10 @@
 //   O  = scale (Qd S + Aqk D)                               (S6, inter + intra chunk)
 //   S <- diag(e^Gl) S + Kt^T D                              (S7)
 //
+// When some channel decays too fast for one anchor per chunk (more than 2^-50 over 16 rows),
+// the chunk's decayed blocks are formed instead with one anchor per 16 rows (the sub-block
+// path); the rest of the chunk is the same.
+//
 // Work split: one 4-CTA cluster per (sequence, head).
 //  * rank 0 ("chain") owns the whole fp32 state (128 x 128) and runs the sequential
 //    part, S5-S7 (and U = T' V), with 128-column MMAs: the dependent-step latency of a
@@ -183,11 +187,11 @@ constexpr uint32_t COL_P1 = 0, COL_W = 64;                                      
 constexpr uint32_t COL_RB = 256;   // prep, sub-block path: one 64-column product per 16-row block
 constexpr uint32_t TMEM_COLS = 512;
 
-// ---- gate range. Per-token log-decays are floored at -10 (alpha >= e^-10 = 4.5e-5): a channel
-// that keeps less than that of its state per token has forgotten it to far below the precision
-// of the bf16 operands either way. A chunk takes the single-anchor path when, on every channel,
-// each 16-row quarter of the chunk decays by less than 2^-50 (so each half by less than
-// 2^-100, which keeps every anchored factor within 2^+-100); otherwise the sub-block path.
+// ---- gate range. A chunk takes the single-anchor path when, on every channel, each 16-row
+// quarter of the chunk decays by less than 2^-50 (so each half by less than 2^-100, which keeps
+// every anchored factor within 2^+-100); otherwise the sub-block path, on which per-token
+// log-decays are floored at -10 (alpha >= e^-10 = 4.5e-5): a channel that keeps less than that of
+// its state per token has forgotten it to far below the precision of the bf16 operands either way.
 constexpr float kFloorLog2 = -14.426950408889634f;   // log2(e^-10)
 constexpr float kQuarterRangeLog2 = 50.f;
 
