@@ -1127,7 +1127,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     // quarter decays beyond the single anchor's range" with the abort flag; only when
                     // that is set does a second barrier tell the two apart
                     const bool unsafe = !(qsum.x >= -kQuarterRangeLog2) || !(qsum.y >= -kQuarterRangeLog2);
-                    if (named_bar_any(2, 256, unsafe || *abort_flag != 0)) {
+                    if (__builtin_expect(named_bar_any(2, 256, unsafe || *abort_flag != 0), 0)) {
                         if (named_bar_any(2, 256, *abort_flag != 0)) break;
                         robust = true;
                         // the sub-block path floors the gates: again with the floored sums
@@ -1145,7 +1145,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int q = 0; q < 4; ++q) qs[q] = *reinterpret_cast<const float2 *>(gq + q * 128 + c0);
                     const float2 ga = f2_add(qs[0], qs[1]);                  // G at the anchor row 31
                     const float2 gl = f2_add(ga, f2_add(qs[2], qs[3]));      // G at row 63
-                    if (robust) {
+                    if (__builtin_expect(robust, 0)) {
                         // ---- sub-block path, part 1 (this thread's rows and channels): the running
                         // log-decay G over the chunk, written over g in the staging tile for the factor
                         // phase, Kt = K 2^(Gl - G) (<= 1), e^Gl; the anchored factors are not used.
@@ -1240,7 +1240,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     }   // single-anchor path
                 }
-                if (robust) {
+                if (__builtin_expect(robust, 0)) {
                     // ---- sub-block path, part 2: the decayed blocks by 16-row block R, each with its own
                     // anchor row a_R = 16R + 7:
                     //   left  (A operand rows, all R):  [K; Q] 2^(G - G_aR)     rows of block R
@@ -1301,7 +1301,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // phase writing their operands (no hop through another warp).
                 if (t == 0) {
                     tc_fence_after();
-                    if (!robust) {
+                    if (__builtin_expect(!robust, 1)) {
                         mbar_arrive(BAR(PB_STAGE_FREE));
                         // [Kh; Qh] Kc^T : A = Kh^T | Qh^T (MN-major, 64-row blocks 16 KB apart), B = Kc^T
                         for (int ks = 0; ks < 8; ++ks)
@@ -1349,51 +1349,46 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                              w4[1], w4[2], w4[3]);
                             }
                     }
-                    uint32_t a[32];
-                    if (!robust) {
-                        tmem_ld32(tmem + lane_base + COL_P1 + half * 32, a);
-                        tmem_wait_ld();
-                    } else {
-                        // row lrow belongs to block (lrow & 63) >> 4, whose product holds it: lanes 0-15 of
-                        // this warp read one product, lanes 16-31 the next
-                        const uint32_t col = COL_RB + 64u * static_cast<uint32_t>(2 * (q4 & 1)) + half * 32;
-                        uint32_t b[32];
+                    // the products' rows: on the common path one 32-column load per thread; on the
+                    // sub-block path row lrow lives in the product of its block (lrow & 63) >> 4, so
+                    // lanes 0-15 and 16-31 of a warp take it from two products, one pass each
+                    const int npass = robust ? 2 : 1;
+                    for (int pass = 0; pass < npass; ++pass) {
+                        uint32_t a[32];
+                        const uint32_t col = robust ? COL_RB + 64u * static_cast<uint32_t>(2 * (q4 & 1) + pass) + half * 32
+                                                    : COL_P1 + half * 32;
                         tmem_ld32(tmem + lane_base + col, a);
-                        tmem_ld32(tmem + lane_base + col + 64, b);
                         tmem_wait_ld();
-                        if (lane >= 16) {
+                        if (t == 0) KDA_TRACE_POINT(m, 27);
+                        if (robust && (lane >> 4) != pass) continue;
+                        if (lrow < 64) {
+                            const int rr = lrow;
+                            const float br = beta_s[rr];
+                            float *rowp = wsf + PR_AKK / 4 + rr * AKK_LD + half * 32;
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) a[i] = b[i];
-                        }
-                    }
-                    if (t == 0) KDA_TRACE_POINT(m, 27);
-                    if (lrow < 64) {
-                        const int rr = lrow;
-                        const float br = beta_s[rr];
-                        float *rowp = wsf + PR_AKK / 4 + rr * AKK_LD + half * 32;
+                            for (int j = 0; j < 8; ++j) {
+                                float v4[4];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            float v4[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int i = half * 32 + 4 * j + e;
-                                v4[e] = i < rr ? br * __uint_as_float(a[4 * j + e]) : 0.f;
+                                for (int e = 0; e < 4; ++e) {
+                                    const int i = half * 32 + 4 * j + e;
+                                    v4[e] = i < rr ? br * __uint_as_float(a[4 * j + e]) : 0.f;
+                                }
+                                *reinterpret_cast<float4 *>(rowp + 4 * j) = make_float4(v4[0], v4[1], v4[2], v4[3]);
                             }
-                            *reinterpret_cast<float4 *>(rowp + 4 * j) = make_float4(v4[0], v4[1], v4[2], v4[3]);
-                        }
-                    } else {
-                        const int rr = lrow - 64;
+                        } else {
+                            const int rr = lrow - 64;
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            float v8[8];
+                            for (int j = 0; j < 4; ++j) {
+                                float v8[8];
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const int i = half * 32 + 8 * j + e;
-                                v8[e] = i <= rr ? __uint_as_float(a[8 * j + e]) : 0.f;
+                                for (int e = 0; e < 8; ++e) {
+                                    const int i = half * 32 + 8 * j + e;
+                                    v8[e] = i <= rr ? __uint_as_float(a[8 * j + e]) : 0.f;
+                                }
+                                const int jj = half * 4 + j;
+                                st_shared_v4(sbase + PR_AVT + sw128(64 + rr, jj), pack_f16(v8[0], v8[1]),
+                                             pack_f16(v8[2], v8[3]), pack_f16(v8[4], v8[5]), pack_f16(v8[6], v8[7]));
                             }
-                            const int jj = half * 4 + j;
-                            st_shared_v4(sbase + PR_AVT + sw128(64 + rr, jj), pack_f16(v8[0], v8[1]),
-                                         pack_f16(v8[2], v8[3]), pack_f16(v8[4], v8[5]), pack_f16(v8[6], v8[7]));
                         }
                     }
                     // blocks of T read as zeros by the fixed-length products below
@@ -1419,7 +1414,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         for (int r = 0; r < 16; ++r) T[(16 * wb + r) * AKK_LD + 16 * wb + li] = x[r];
                     }
                 }
-                if (robust) {
+                if (__builtin_expect(robust, 0)) {
                     // ---- sub-block path, part 3 (its products have completed): the W and Qd operands
                     // from the chunk-start-relative factors, K 2^G and Q 2^G (<= 1), over the left factors
                     // (the scale e^Ga applied to them later is 1 on this path); the T' rows of the
@@ -1450,7 +1445,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (named_bar_any(2, 256, *abort_flag != 0)) break;
                 if (t == 0) {
                     mbar_arrive(BAR(PB_OUTA_READY));
-                    if (robust) mbar_arrive(BAR(PB_STAGE_FREE));   // q, k and G have been read
+                    if (__builtin_expect(robust, 0)) mbar_arrive(BAR(PB_STAGE_FREE));   // q, k and G have been read
                     KDA_TRACE_POINT(m, 9);
                 }
 
