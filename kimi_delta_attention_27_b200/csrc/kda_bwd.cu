@@ -136,11 +136,19 @@ __device__ void load_chunk(const BwdParams &p, const Unit &u, int64_t t0, int L,
         const int r = t >> 4, c0 = (t & 15) * 8;
         const size_t off = ((static_cast<size_t>(t0) + r) * H + u.h) * D + c0;
         if (r < L) {
+            // 16-byte loads: 8 bf16 of k and of q, 2 x 4 fp32 of g (rows start 256 / 512 B apart)
+            const uint4 kw = *reinterpret_cast<const uint4 *>(p.k + off);
+            const uint4 qw = *reinterpret_cast<const uint4 *>(p.q + off);
+            const float4 g0 = *reinterpret_cast<const float4 *>(p.g + off);
+            const float4 g1 = *reinterpret_cast<const float4 *>(p.g + off + 4);
+            const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, qq[4] = {qw.x, qw.y, qw.z, qw.w};
+            const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                sm[SM_K + r * DP + c0 + e] = bf(p.k[off + e]);
-                sm[SM_Q + r * DP + c0 + e] = bf(p.q[off + e]);
-                sm[SM_G + r * DP + c0 + e] = fmaxf(p.g[off + e] * kLog2e, kFloorLog2);
+                const uint32_t kb2 = kk[e >> 1], qb2 = qq[e >> 1];
+                sm[SM_K + r * DP + c0 + e] = __uint_as_float((e & 1) ? (kb2 & 0xFFFF0000u) : (kb2 << 16));
+                sm[SM_Q + r * DP + c0 + e] = __uint_as_float((e & 1) ? (qb2 & 0xFFFF0000u) : (qb2 << 16));
+                sm[SM_G + r * DP + c0 + e] = fmaxf(gg[e] * kLog2e, kFloorLog2);
             }
         } else {
 #pragma unroll
@@ -150,15 +158,16 @@ __device__ void load_chunk(const BwdParams &p, const Unit &u, int64_t t0, int L,
     {   // V and dO slices: thread t takes row t >> 4, columns 2 (t & 15) .. + 2 of the slice
         const int r = t >> 4, j0 = (t & 15) * 2;
         const size_t off = ((static_cast<size_t>(t0) + r) * H + u.h) * D + u.vs * VS + j0;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            float v = 0.f, dO = 0.f;
-            if (r < L) {
-                v = bf(p.v[off + e]);
-                if (with_do) dO = bf(p.dout[off + e]);
-            }
-            sm[SM_V + r * VP + j0 + e] = v;
-            if (with_do) sm[SM_DO + r * VP + j0 + e] = dO;
+        uint32_t vw = 0u, dw = 0u;   // two bf16 each
+        if (r < L) {
+            vw = *reinterpret_cast<const uint32_t *>(p.v + off);
+            if (with_do) dw = *reinterpret_cast<const uint32_t *>(p.dout + off);
+        }
+        sm[SM_V + r * VP + j0] = __uint_as_float(vw << 16);
+        sm[SM_V + r * VP + j0 + 1] = __uint_as_float(vw & 0xFFFF0000u);
+        if (with_do) {
+            sm[SM_DO + r * VP + j0] = __uint_as_float(dw << 16);
+            sm[SM_DO + r * VP + j0 + 1] = __uint_as_float(dw & 0xFFFF0000u);
         }
     }
     if (t < CB) {
