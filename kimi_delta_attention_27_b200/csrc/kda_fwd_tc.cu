@@ -63,8 +63,8 @@ __device__ int g_kda_test_skip_chunk = -1;
 #ifdef KDA_TRACE
 // Development-only timeline: when built with -DKDA_TRACE, the first cluster
 // records %globaltimer at fixed points per chunk into g_kda_trace
-// [rank][chunk < 64][point < 32]. The product build compiles none of this.
-__device__ unsigned long long g_kda_trace[4 * 64 * 32];
+// [rank][chunk < 64][point < 48]. The product build compiles none of this.
+__device__ unsigned long long g_kda_trace[4 * 64 * 48];
 // per cluster: chain CTA start, end, SM id, then the SM ids of ranks 1-3 and the ring address
 __device__ unsigned long long g_kda_cluster_trace[1024 * 8];
 #define KDA_TRACE_CLUSTER(slot, value)                                                              \
@@ -77,7 +77,7 @@ __device__ unsigned long long g_kda_cluster_trace[1024 * 8];
 #define KDA_TRACE_POINT(chunk, point)                                                               \
     do {                                                                                            \
         if (blockIdx.x / 4 == KDA_TRACE_CLUSTER_ID && (chunk) < 64)                                 \
-            g_kda_trace[(rank * 64 + (chunk)) * 32 + (point)] = ptx::globaltimer();                 \
+            g_kda_trace[(rank * 64 + (chunk)) * 48 + (point)] = ptx::globaltimer();                 \
     } while (0)
 #else
 #define KDA_TRACE_CLUSTER(slot, value) \
@@ -231,6 +231,22 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 __device__ __forceinline__ float bf2f(uint16_t x) { return __uint_as_float(static_cast<uint32_t>(x) << 16); }
 __device__ __forceinline__ float lo_bf(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float hi_bf(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// fp32 -> tf32 (round to nearest, ties away from zero), the operand format of the tf32 MMA
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// d (16 x 8, fp32) += a (16 x 8, tf32, row-major) * b (8 x 8, tf32), one warp. Fragments, with
+// g = lane / 4 and i = lane % 4: a = {(g, i), (g + 8, i), (g, i + 4), (g + 8, i + 4)},
+// b = {(i, g), (i + 4, g)}, d = {(g, 2i), (g, 2i + 1), (g + 8, 2i), (g + 8, 2i + 1)}.
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -594,9 +610,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // ---- intra-chunk output product, C1^T[:, 64..127] += D^T Aqk^T, issued once C3^T
             // (the other reader of D^T, on the critical path) has completed
             for (int n = 0; n < nch; ++n) {
-                if (!wait_bar(BAR(CB_C3_FULL), n & 1, abort_flag)) break;
+                if (!__all_sync(0xffffffffu, wait_bar(BAR(CB_C3_FULL), n & 1, abort_flag))) break;
                 tc_fence_after();
-                if (lane == 0) {
+                if (elect_one()) {
                     const uint32_t slot = sbase + CH_SLOT + (n & 1) * SET_STRIDE;
                     for (int ks = 0; ks < 4; ++ks)
                         mma_f16_ts(tmem + COL_C1 + (n & 1) * 128 + 64, tmem + COL_DT + ks * 8,
@@ -651,51 +667,62 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tmem_st32(tmem + lane_base + COL_SP + 32 * half, w);
                 tmem_wait_st();
             };
-            // The products are issued by one thread (tid 128, a D^T warp) as soon as their operands
-            // are in place (a named barrier among the writers), with no hop through another warp.
+            // The products are issued by warp 4 (a D^T warp) as soon as their operands are in place
+            // (a named barrier among the writers), with no hop through another warp: the warp enters
+            // converged and one elected lane issues, so that the operands stay warp-uniform.
             // value-side product of chunk n into its C1^T buffer (no state involved); C1^T has two
             // buffers, so chunk n's buffer was last read in chunk n - 2
             auto issue_uv = [&](int n) -> bool {
                 const int s1 = n & 1;
                 const uint32_t slot = sbase + CH_SLOT + s1 * SET_STRIDE;
-                if (!wait_bar(BAR(CB_FULL + s1), (n >> 1) & 1, abort_flag)) return false;
+                // the lanes agree on the outcome before the election
+                if (!__all_sync(0xffffffffu, wait_bar(BAR(CB_FULL + s1), (n >> 1) & 1, abort_flag))) return false;
                 tc_fence_after();
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tmem + COL_C1 + s1 * 128, smem_desc(slot + SET_V + ks * 2048, 8192, 1024, kSwizzle128),
-                            smem_desc(slot + SET_T + ks * 32, 16, 1024, kSwizzle128), ID_UVT, ks > 0);
+                if (elect_one()) {
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(tmem + COL_C1 + s1 * 128, smem_desc(slot + SET_V + ks * 2048, 8192, 1024, kSwizzle128),
+                                smem_desc(slot + SET_T + ks * 32, 16, 1024, kSwizzle128), ID_UVT, ks > 0);
+                }
+                __syncwarp();
                 return true;
             };
             auto issue_state = [&](int n) {
                 const int s1 = n & 1;
                 const uint32_t slot = sbase + CH_SLOT + s1 * SET_STRIDE;
                 tc_fence_after();
-                KDA_TRACE_POINT(n, 13);
-                // first K step in two halves: columns 0..63 accumulate onto U^T, columns 64..127
-                // (the output half, not touched by the value-side product) start from zero
-                mma_f16_ts(tmem + COL_C1 + s1 * 128, tmem + COL_SP, smem_desc(slot + SET_W, 16384, 1024, kSwizzle128),
-                           ID_STATE_H, 1);
-                mma_f16_ts(tmem + COL_C1 + s1 * 128 + 64, tmem + COL_SP,
-                           smem_desc(slot + SET_Q, 16384, 1024, kSwizzle128), ID_STATE_H, 0);
-                for (int ks = 1; ks < 8; ++ks)
-                    mma_f16_ts(tmem + COL_C1 + s1 * 128, tmem + COL_SP + ks * 8,
-                               smem_desc(slot + SET_W + ks * 2048, 16384, 1024, kSwizzle128), ID_STATE_T, 1);
-                mma_commit(BAR(CB_C1_FULL));
-                KDA_TRACE_POINT(n, 3);
+                if (elect_one()) {
+                    KDA_TRACE_POINT(n, 13);
+                    // first K step in two halves: columns 0..63 accumulate onto U^T, columns 64..127
+                    // (the output half, not touched by the value-side product) start from zero
+                    mma_f16_ts(tmem + COL_C1 + s1 * 128, tmem + COL_SP,
+                               smem_desc(slot + SET_W, 16384, 1024, kSwizzle128), ID_STATE_H, 1);
+                    mma_f16_ts(tmem + COL_C1 + s1 * 128 + 64, tmem + COL_SP,
+                               smem_desc(slot + SET_Q, 16384, 1024, kSwizzle128), ID_STATE_H, 0);
+                    for (int ks = 1; ks < 8; ++ks)
+                        mma_f16_ts(tmem + COL_C1 + s1 * 128, tmem + COL_SP + ks * 8,
+                                   smem_desc(slot + SET_W + ks * 2048, 16384, 1024, kSwizzle128), ID_STATE_T, 1);
+                    mma_commit(BAR(CB_C1_FULL));
+                    KDA_TRACE_POINT(n, 3);
+                }
+                __syncwarp();
             };
             auto issue_c3 = [&](int n) {
                 const uint32_t slot = sbase + CH_SLOT + (n & 1) * SET_STRIDE;
                 tc_fence_after();
-                KDA_TRACE_POINT(n, 4);
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16_ts(tmem + COL_C3, tmem + COL_DT + ks * 8,
-                               smem_desc(slot + SET_KT + ks * 32, 16, 1024, kSwizzle128), ID_C3T, ks > 0);
-                mma_commit(BAR(CB_C3_FULL));
-                KDA_TRACE_POINT(n, 5);
+                if (elect_one()) {
+                    KDA_TRACE_POINT(n, 4);
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16_ts(tmem + COL_C3, tmem + COL_DT + ks * 8,
+                                   smem_desc(slot + SET_KT + ks * 32, 16, 1024, kSwizzle128), ID_C3T, ks > 0);
+                    mma_commit(BAR(CB_C3_FULL));
+                    KDA_TRACE_POINT(n, 5);
+                }
+                __syncwarp();
             };
             write_sprime();
             tc_fence_before();
             named_bar_sync(4, 256);
-            if (tid == 128 && nch > 0) {
+            if (warp == 4 && nch > 0) {
                 if (issue_uv(0)) issue_state(0);
             }
             __syncwarp();
@@ -729,10 +756,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (tid == 128) KDA_TRACE_POINT(n, 1);
                     tc_fence_before();
                     named_bar_sync(3, 128);
-                    if (tid == 128) {
+                    if (warp == 4) {
                         issue_c3(n);
                         // the next chunk's value-side product follows on the tensor pipe; this
-                        // thread waits for its slot here, so that the product runs during the C3^T
+                        // warp waits for its slot here, so that the product runs during the C3^T
                         // epilogue rather than ahead of the next state product
                         if (n + 1 < nch) ok = issue_uv(n + 1);
                     }
@@ -773,7 +800,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (lane == 0) mbar_arrive(BAR(CB_SFREE + sl));   // decay reads done
                 if (n + 1 < nch) {
                     if (named_bar_any(4, 256, *abort_flag != 0)) break;
-                    if (tid == 128) issue_state(n + 1);
+                    if (warp == 4) issue_state(n + 1);
                     __syncwarp();
                 }
                 if (tid == 128) KDA_TRACE_POINT(n, 11);
@@ -1060,9 +1087,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const float *beta_s = reinterpret_cast<const float *>(miscg + M_BETAQ) + (kk & 1) * C;
 #ifdef KDA_TRACE
                 if (t == 0 && blockIdx.x / 4 == KDA_TRACE_CLUSTER_ID && m < 64) {
-                    g_kda_trace[(rank * 64 + m) * 32 + 0] = trace_start;
-                    g_kda_trace[(rank * 64 + m) * 32 + 25] = trace_afree;
-                    g_kda_trace[(rank * 64 + m) * 32 + 26] = trace_sfull;
+                    g_kda_trace[(rank * 64 + m) * 48 + 0] = trace_start;
+                    g_kda_trace[(rank * 64 + m) * 48 + 25] = trace_afree;
+                    g_kda_trace[(rank * 64 + m) * 48 + 26] = trace_sfull;
                 }
 #endif
                 if (t == 0) KDA_TRACE_POINT(m, 1);
@@ -1140,6 +1167,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         *reinterpret_cast<float2 *>(gq + tq * 128 + c0) = f2_add(sp[0], sp[1]);
                         if (named_bar_any(2, 256, *abort_flag != 0)) break;
                     }
+                    if (t == 0) KDA_TRACE_POINT(m, 30);
                     float2 qs[4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) qs[q] = *reinterpret_cast<const float2 *>(gq + q * 128 + c0);
@@ -1239,6 +1267,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         *reinterpret_cast<float2 *>(ega_s + c0) = make_float2(ex2_approx(ga.x), ex2_approx(ga.y));
                     }
                     }   // single-anchor path
+                    if (t == 0) KDA_TRACE_POINT(m, 31);
                 }
                 if (__builtin_expect(robust, 0)) {
                     // ---- sub-block path, part 2: the decayed blocks by 16-row block R, each with its own
@@ -1297,29 +1326,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 fence_proxy_async_smem();
                 if (named_bar_any(2, 256, *abort_flag != 0)) break;
-                // The prep MMAs are issued by this thread right after the barrier that ends the
-                // phase writing their operands (no hop through another warp).
-                if (t == 0) {
+                // The prep MMAs are issued by warp 4 right after the barrier that ends the phase
+                // writing their operands (no hop through another warp); one elected lane issues.
+                if (warp == 4) {
                     tc_fence_after();
-                    if (__builtin_expect(!robust, 1)) {
-                        mbar_arrive(BAR(PB_STAGE_FREE));
-                        // [Kh; Qh] Kc^T : A = Kh^T | Qh^T (MN-major, 64-row blocks 16 KB apart), B = Kc^T
-                        for (int ks = 0; ks < 8; ++ks)
-                            mma_f16(tmem + COL_P1, smem_desc(sbase + PR_KH + ks * 2048, 16384, 1024, kSwizzle128),
-                                    smem_desc(sbase + PR_KC + ks * 2048, 16384, 1024, kSwizzle128), ID_P1, ks > 0);
-                    } else {
-                        // the staging tile is still read after these products (G, q, k)
-#pragma unroll
-                        for (int R = 0; R < 4; ++R) {
-                            const uint32_t rt = sbase + (R == 0 ? PR_KC : R == 1 ? PR_AKK : R == 2 ? PR_T : PR_AVT);
+                    if (elect_one()) {
+                        if (__builtin_expect(!robust, 1)) {
+                            mbar_arrive(BAR(PB_STAGE_FREE));
+                            // [Kh; Qh] Kc^T : A = Kh^T | Qh^T (MN-major, 64-row blocks 16 KB apart), B = Kc^T
                             for (int ks = 0; ks < 8; ++ks)
-                                mma_f16(tmem + COL_RB + 64 * R,
-                                        smem_desc(sbase + PR_KH + ks * 2048, 16384, 1024, kSwizzle128),
-                                        smem_desc(rt + ks * 2048, 16384, 1024, kSwizzle128), ID_P1, ks > 0);
+                                mma_f16(tmem + COL_P1, smem_desc(sbase + PR_KH + ks * 2048, 16384, 1024, kSwizzle128),
+                                        smem_desc(sbase + PR_KC + ks * 2048, 16384, 1024, kSwizzle128), ID_P1, ks > 0);
+                        } else {
+                            // the staging tile is still read after these products (G, q, k)
+#pragma unroll
+                            for (int R = 0; R < 4; ++R) {
+                                const uint32_t rt = sbase + (R == 0 ? PR_KC : R == 1 ? PR_AKK : R == 2 ? PR_T : PR_AVT);
+                                for (int ks = 0; ks < 8; ++ks)
+                                    mma_f16(tmem + COL_RB + 64 * R,
+                                            smem_desc(sbase + PR_KH + ks * 2048, 16384, 1024, kSwizzle128),
+                                            smem_desc(rt + ks * 2048, 16384, 1024, kSwizzle128), ID_P1, ks > 0);
+                            }
                         }
+                        mma_commit(BAR(PB_P1_DONE));
+                        KDA_TRACE_POINT(m, 2);
                     }
-                    mma_commit(BAR(PB_P1_DONE));
-                    KDA_TRACE_POINT(m, 2);
+                    __syncwarp();
                 }
                 // value tile bf16 -> fp16 in place (B operand of the value-side MMA)
                 wait_bar(BAR(PB_VSTAGE_FULL), kk & 1, abort_flag);
@@ -1391,6 +1423,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             }
                         }
                     }
+                    if (t == 0) KDA_TRACE_POINT(m, 32);
                     // blocks of T read as zeros by the fixed-length products below
                     float *T = wsf + PR_T / 4;
                     T[(t >> 4) * AKK_LD + 16 + (t & 15)] = 0.f;               // rows 0-15, cols 16-31
@@ -1454,11 +1487,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 //       S2 epilogue, by the warps that wrote those blocks of A),
                 //   (b) the two 16 x 16 blocks below them inside each 32 x 32 diagonal block,
                 //   (c) the 32 x 32 block below the diagonal,
-                // each off-diagonal block as  T_IJ = -T_II (A_IJ T_JJ).
+                // each off-diagonal block as  T_IJ = -T_II (A_IJ T_JJ). The products of (b) and (c)
+                // are warp-level tf32 MMAs (m16n8k8) on operands read straight from the fp32 tiles:
+                // a warp owns a 16 x 8 tile of the result, so each operand element is read by a
+                // few lanes instead of once per output column.
                 {
                     const float *A = wsf + PR_AKK / 4;
                     float *T = wsf + PR_T / 4;
-                    float *P = wsf + PR_P / 4;
+                    float *P = wsf + PR_P / 4;   // 8 tiles of 16 x 8 floats (row stride 8)
                     if (t == 0) KDA_TRACE_POINT(m, 10);
                     // T' = T diag(beta) is written straight into its two operand tiles as each block of
                     // T becomes final: fp16 (rows 0..63 of the [T'; Aqk] tile) and bf16 (TB); the blocks
@@ -1468,109 +1504,117 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         return base + sw128(static_cast<uint32_t>(r), static_cast<uint32_t>(c >> 3)) +
                                static_cast<uint32_t>(c & 7) * 2u;
                     };
-                    // (b) blocks (1,0) and (3,2): P = A_IJ T_JJ, then T_IJ = -T_II P (two columns per thread)
-                    {
-                        const int blk = t >> 7, rr = (t >> 3) & 15, cc = (t & 7) * 2;
-                        const int J = 2 * blk, I = J + 1;
-                        const float *arow = A + (16 * I + rr) * AKK_LD + 16 * J;
-                        float p0 = 0.f, p1 = 0.f;
+                    const int w8 = warp - 4, g8 = lane >> 2, tg = lane & 3;   // MMA fragment coordinates
+                    // a 16 x 8 A fragment (rows r0 + g8, r0 + g8 + 8; columns c0 + tg, c0 + tg + 4) of a
+                    // row-major fp32 tile with row stride AKK_LD
+                    auto frag_a = [&](const float *M, int r0, int c0, uint32_t (&a)[4]) {
+                        const float *p0 = M + (r0 + g8) * AKK_LD + c0 + tg;
+                        a[0] = to_tf32(p0[0]);
+                        a[1] = to_tf32(p0[8 * AKK_LD]);
+                        a[2] = to_tf32(p0[4]);
+                        a[3] = to_tf32(p0[8 * AKK_LD + 4]);
+                    };
+                    // an 8 x 8 B fragment (rows k0 + tg, k0 + tg + 4; column n0 + g8) of a row-major tile
+                    auto frag_b = [&](const float *M, int ld, int k0, int n0, uint32_t (&b)[2]) {
+                        b[0] = to_tf32(M[(k0 + tg) * ld + n0 + g8]);
+                        b[1] = to_tf32(M[(k0 + tg + 4) * ld + n0 + g8]);
+                    };
+                    // T' (= -acc diag(beta)) of the 16 x 8 result tile at rows r0, columns n0
+                    auto store_tprime = [&](const float (&acc)[4], int r0, int n0) {
+                        const int c = n0 + 2 * tg;
+                        const float b0 = -beta_s[c], b1 = -beta_s[c + 1];
 #pragma unroll
-                        for (int j4 = 0; j4 < 4; ++j4) {
-                            const float4 av = *reinterpret_cast<const float4 *>(arow + 4 * j4);
-                            const float a4[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 tv =
-                                    *reinterpret_cast<const float2 *>(T + (16 * J + 4 * j4 + e) * AKK_LD + 16 * J + cc);
-                                p0 = fmaf(a4[e], tv.x, p0);
-                                p1 = fmaf(a4[e], tv.y, p1);
-                            }
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const float x0 = acc[2 * hh] * b0, x1 = acc[2 * hh + 1] * b1;
+                            st_shared_u32(tp_addr(sbase + PR_AVT, r0 + g8 + 8 * hh, c), pack_f16(x0, x1));
+                            st_shared_u32(tp_addr(sbase + PR_TB, r0 + g8 + 8 * hh, c), pack_bf16(x0, x1));
                         }
-                        *reinterpret_cast<float2 *>(P + blk * 256 + rr * 16 + cc) = make_float2(p0, p1);
-                        // T' of the diagonal blocks (final since (a)): row t >> 2, 4 columns
-                        {
-                            const int r = t >> 2, cq = (t & 3) * 4, c = (r & ~15) + cq;
-                            const float4 tv = *reinterpret_cast<const float4 *>(T + r * AKK_LD + c);
-                            const float4 bv = *reinterpret_cast<const float4 *>(beta_s + c);
-                            const float x0 = tv.x * bv.x, x1 = tv.y * bv.y, x2 = tv.z * bv.z, x3 = tv.w * bv.w;
-                            st_shared_v2(tp_addr(sbase + PR_AVT, r, c), pack_f16(x0, x1), pack_f16(x2, x3));
-                            st_shared_v2(tp_addr(sbase + PR_TB, r, c), pack_bf16(x0, x1), pack_bf16(x2, x3));
-                        }
-                        if (named_bar_any(2, 256, *abort_flag != 0)) break;
-                        if (t == 0) KDA_TRACE_POINT(m, 29);
-                        const float *trow = T + (16 * I + rr) * AKK_LD + 16 * I;
-                        p0 = 0.f;
-                        p1 = 0.f;
+                    };
+                    if (w8 < 4) {
+                        // (b) warp (blk, nt): T_IJ[:, 8 nt .. 8 nt + 7] for I = 2 blk + 1, J = 2 blk
+                        const int blk = w8 >> 1, nt = w8 & 1, I = 2 * blk + 1, J = 2 * blk;
+                        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int j4 = 0; j4 < 4; ++j4) {
-                            const float4 tv4 = *reinterpret_cast<const float4 *>(trow + 4 * j4);
-                            const float t4[4] = {tv4.x, tv4.y, tv4.z, tv4.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 pv = *reinterpret_cast<const float2 *>(P + blk * 256 + (4 * j4 + e) * 16 + cc);
-                                p0 = fmaf(t4[e], pv.x, p0);
-                                p1 = fmaf(t4[e], pv.y, p1);
-                            }
+                        for (int ks = 0; ks < 2; ++ks) {   // P = A_IJ T_JJ[:, n-tile]
+                            if (ks < nt) continue;         // T_JJ is lower triangular
+                            uint32_t a[4], b[2];
+                            frag_a(A, 16 * I, 16 * J + 8 * ks, a);
+                            frag_b(T, AKK_LD, 16 * J + 8 * ks, 16 * J + 8 * nt, b);
+                            mma_tf32_16x8x8(acc, a, b);
                         }
-                        *reinterpret_cast<float2 *>(T + (16 * I + rr) * AKK_LD + 16 * J + cc) = make_float2(-p0, -p1);
-                        const int r = 16 * I + rr, c = 16 * J + cc;
-                        const float x0 = -p0 * beta_s[c], x1 = -p1 * beta_s[c + 1];
-                        st_shared_u32(tp_addr(sbase + PR_AVT, r, c), pack_f16(x0, x1));
-                        st_shared_u32(tp_addr(sbase + PR_TB, r, c), pack_bf16(x0, x1));
-                        if (t == 0) KDA_TRACE_POINT(m, 13);
+                        // the product tile becomes the B operand of the next step through this warp's
+                        // own scratch tile
+                        float *Pw = P + w8 * 128;
+                        *reinterpret_cast<float2 *>(Pw + g8 * 8 + 2 * tg) = make_float2(acc[0], acc[1]);
+                        *reinterpret_cast<float2 *>(Pw + (g8 + 8) * 8 + 2 * tg) = make_float2(acc[2], acc[3]);
+                        __syncwarp();
+                        float res[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) {   // T_II P
+                            uint32_t a[4], b[2];
+                            frag_a(T, 16 * I, 16 * I + 8 * ks, a);
+                            frag_b(Pw, 8, 8 * ks, 0, b);
+                            mma_tf32_16x8x8(res, a, b);
+                        }
+                        // T_IJ = -T_II P: fp32 for (c), T' for the products
+                        const int r = 16 * I + g8, c = 16 * J + 8 * nt + 2 * tg;
+                        *reinterpret_cast<float2 *>(T + r * AKK_LD + c) = make_float2(-res[0], -res[1]);
+                        *reinterpret_cast<float2 *>(T + (r + 8) * AKK_LD + c) = make_float2(-res[2], -res[3]);
+                        store_tprime(res, 16 * I, 16 * J + 8 * nt);
+                    } else {
+                        // T' of the four diagonal blocks (final since (a)): 128 threads, one row and 8
+                        // columns each
+                        const int tt = t - 128, r = tt >> 1, c = (r & ~15) + 8 * (tt & 1);
+                        const float4 t0 = *reinterpret_cast<const float4 *>(T + r * AKK_LD + c);
+                        const float4 t1 = *reinterpret_cast<const float4 *>(T + r * AKK_LD + c + 4);
+                        const float4 b0 = *reinterpret_cast<const float4 *>(beta_s + c);
+                        const float4 b1 = *reinterpret_cast<const float4 *>(beta_s + c + 4);
+                        const float x[8] = {t0.x * b0.x, t0.y * b0.y, t0.z * b0.z, t0.w * b0.w,
+                                            t1.x * b1.x, t1.y * b1.y, t1.z * b1.z, t1.w * b1.w};
+                        st_shared_v4(tp_addr(sbase + PR_AVT, r, c), pack_f16(x[0], x[1]), pack_f16(x[2], x[3]),
+                                     pack_f16(x[4], x[5]), pack_f16(x[6], x[7]));
+                        st_shared_v4(tp_addr(sbase + PR_TB, r, c), pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                                     pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
                     }
+                    if (t == 0) KDA_TRACE_POINT(m, 13);
                     if (named_bar_any(2, 256, *abort_flag != 0)) break;
                     if (t == 0) KDA_TRACE_POINT(m, 11);
-                    // (c) rows 32..63, columns 0..31: P2 = A[32:, :32] T[:32, :32]; T = -T[32:, 32:] P2.
-                    // Lane = row, warp = 4-column group, so the T and P2 reads are warp-uniform
-                    // (broadcast) and the zero block T[0:16, 16:32] is skipped by whole warps. P2 is
-                    // stored with its 16-byte groups XOR-swizzled by row to keep the stores conflict-free.
-                    // A warp reads back only the P2 columns it wrote, so it waits for no other warp.
+                    // (c) warp (mt, nt): rows 32 + 16 mt .. + 15, columns 8 nt .. 8 nt + 7 of
+                    //   P2 = A[32:, :32] T[:32, :32],  T[32:, :32] = -T[32:, 32:] P2.
+                    // T[:32, :32] is lower triangular, so the n-tile nt needs k-steps nt .. 3 only;
+                    // T[32:48, 48:64] is zero, so rows 32..47 need P2 rows 0..15 (their own tile) and
+                    // rows 48..63 wait for that tile from the warp of the same nt (barrier 5 + nt).
                     {
-                        const int rr = t & 31, c4 = (t >> 5) * 4;
-                        const float *arow = A + (32 + rr) * AKK_LD;
-                        float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-                        const int j4lo = c4 >= 16 ? 4 : 0;
+                        const int mt = w8 >> 2, nt = w8 & 3;
+                        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int j4 = 0; j4 < 8; ++j4) {
-                            if (j4 < j4lo) continue;
-                            const float4 av = *reinterpret_cast<const float4 *>(arow + 4 * j4);
-                            const float a4[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float4 tv = *reinterpret_cast<const float4 *>(T + (4 * j4 + e) * AKK_LD + c4);
-                                p0 = fmaf(a4[e], tv.x, p0);
-                                p1 = fmaf(a4[e], tv.y, p1);
-                                p2 = fmaf(a4[e], tv.z, p2);
-                                p3 = fmaf(a4[e], tv.w, p3);
-                            }
+                        for (int ks = 0; ks < 4; ++ks) {
+                            if (ks < nt) continue;
+                            uint32_t a[4], b[2];
+                            frag_a(A, 32 + 16 * mt, 8 * ks, a);
+                            frag_b(T, AKK_LD, 8 * ks, 8 * nt, b);
+                            mma_tf32_16x8x8(acc, a, b);
                         }
-                        *reinterpret_cast<float4 *>(P + rr * 32 + (((c4 >> 2) ^ (rr & 7)) << 2)) =
-                            make_float4(p0, p1, p2, p3);
+                        float *Pw = P + w8 * 128;   // P2 rows 16 mt .. 16 mt + 15, columns of n-tile nt
+                        *reinterpret_cast<float2 *>(Pw + g8 * 8 + 2 * tg) = make_float2(acc[0], acc[1]);
+                        *reinterpret_cast<float2 *>(Pw + (g8 + 8) * 8 + 2 * tg) = make_float2(acc[2], acc[3]);
+                        if (mt == 0) {
+                            named_bar_arrive(5 + nt, 64);   // the tile is written: rows 48..63 may read it
+                        } else {
+                            named_bar_sync(5 + nt, 64);
+                        }
                         __syncwarp();
-                        if (t == 0) KDA_TRACE_POINT(m, 14);
-                        const float *trow = T + (32 + rr) * AKK_LD + 32;
-                        p0 = p1 = p2 = p3 = 0.f;
+                        float res[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int j4 = 0; j4 < 8; ++j4) {
-                            const float4 tv4 = *reinterpret_cast<const float4 *>(trow + 4 * j4);
-                            const float t4[4] = {tv4.x, tv4.y, tv4.z, tv4.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = 4 * j4 + e;
-                                const float4 pv =
-                                    *reinterpret_cast<const float4 *>(P + j * 32 + (((c4 >> 2) ^ (j & 7)) << 2));
-                                p0 = fmaf(t4[e], pv.x, p0);
-                                p1 = fmaf(t4[e], pv.y, p1);
-                                p2 = fmaf(t4[e], pv.z, p2);
-                                p3 = fmaf(t4[e], pv.w, p3);
-                            }
+                        for (int ks = 0; ks < 4; ++ks) {
+                            if (mt == 0 && ks >= 2) continue;
+                            uint32_t a[4], b[2];
+                            frag_a(T, 32 + 16 * mt, 32 + 8 * ks, a);
+                            frag_b(P + ((ks >> 1) * 4 + nt) * 128, 8, 8 * (ks & 1), 0, b);
+                            mma_tf32_16x8x8(res, a, b);
                         }
                         // final block of T; T itself is not read again, only T' is written
-                        const float4 bv = *reinterpret_cast<const float4 *>(beta_s + c4);
-                        const float x0 = -p0 * bv.x, x1 = -p1 * bv.y, x2 = -p2 * bv.z, x3 = -p3 * bv.w;
-                        st_shared_v2(tp_addr(sbase + PR_AVT, 32 + rr, c4), pack_f16(x0, x1), pack_f16(x2, x3));
-                        st_shared_v2(tp_addr(sbase + PR_TB, 32 + rr, c4), pack_bf16(x0, x1), pack_bf16(x2, x3));
+                        store_tprime(res, 32 + 16 * mt, 8 * nt);
                     }
                     if (t == 0) KDA_TRACE_POINT(m, 12);
                 }
@@ -1578,14 +1622,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 fence_proxy_async_smem();
                 if (t == 0) KDA_TRACE_POINT(m, 17);
                 if (named_bar_any(2, 256, *abort_flag != 0)) break;
-                if (t == 0) {
+                if (warp == 4) {
                     tc_fence_after();
-                    // W'^T = Kh^T T'^T (bf16)
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tmem + COL_W, smem_desc(sbase + PR_KH + ks * 32, 16, 1024, kSwizzle128),
-                                smem_desc(sbase + PR_TB + ks * 32, 16, 1024, kSwizzle128), ID_W, ks > 0);
-                    mma_commit(BAR(PB_WAV_DONE));
-                    KDA_TRACE_POINT(m, 4);
+                    if (elect_one()) {
+                        // W'^T = Kh^T T'^T (bf16)
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_f16(tmem + COL_W, smem_desc(sbase + PR_KH + ks * 32, 16, 1024, kSwizzle128),
+                                    smem_desc(sbase + PR_TB + ks * 32, 16, 1024, kSwizzle128), ID_W, ks > 0);
+                        mma_commit(BAR(PB_WAV_DONE));
+                        KDA_TRACE_POINT(m, 4);
+                    }
+                    __syncwarp();
                 }
                 // -------- Qd = Q e^G = Qh diag(e^Ga) (bf16, over the dead A workspace) while W' runs
                 {
