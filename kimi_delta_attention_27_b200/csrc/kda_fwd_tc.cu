@@ -1104,7 +1104,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const bool flip = (lane >> 2) & 1;
                 bool robust = false;   // this chunk takes the sub-block path (CTA-uniform)
                 {
-                    const int grp = (warp - 4) & 3;
+                    // the two half-warps take channel groups of different parity, so that their
+                    // bf16-pair loads of q and k (rows 16 apart) fall on disjoint banks
+                    const int grp = ((warp - 4) & 3) ^ (lane >> 4);
                     const int cp = grp * 16 + (lane & 15);
                     const int tq = 2 * ((warp - 4) >> 2) + (lane >> 4);
                     const int c0 = 2 * cp, r0 = 16 * tq;
@@ -1370,7 +1372,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (t == 0) KDA_TRACE_POINT(m, 3);
                 {
                     {
-                        const int cp = ((warp - 4) & 3) * 16 + (lane & 15);
+                        const int cp = (((warp - 4) & 3) ^ (lane >> 4)) * 16 + (lane & 15);   // as in S1
                         const int tq = 2 * ((warp - 4) >> 2) + (lane >> 4);
 #pragma unroll
                         for (int ch = 0; ch < 2; ++ch)
