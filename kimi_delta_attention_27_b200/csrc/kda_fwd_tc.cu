@@ -143,7 +143,7 @@ constexpr uint32_t M_BETA = 256, M_EGA = 512;                  // 64, 128 floats
 // prep: beta of the two staged chunks (2 x 64 floats), the chunk index of the last four local
 // chunks, the number of chunks the chain CTA has pulled (written by the chain CTA);
 // chain: the next chunk to hand out (incremented by the prep CTAs)
-constexpr uint32_t M_BETAQ = 1024, M_CHUNKQ = 1536, M_CONSUMED = 1552, M_NEXT = 1568;
+constexpr uint32_t M_BETAQ = 1024, M_CHUNKQ = 1536, M_CONSUMED = 1552, M_NEXT = 1568;   // the last two: chain
 constexpr uint32_t M_DEC = 2048;                               // 2 x 128 floats (e^Gl, part of the set)
 constexpr uint32_t M_TMEM = 3072, M_ABORT = 3088, M_SMID = 3104;
 constexpr uint32_t M_HTINFO = 3136;   // chain: where the final state goes (pointer, offset, flags)
@@ -175,8 +175,7 @@ enum {
     PB_OUTC_READY,      // Qd^T (over A), T' and Aqk, V, e^Gl final
     PB_OUTA_FREE,       // publisher has read part A out
     PB_OUTC_FREE,       // publisher has read part C out
-    PB_RING_FREE = 15,  // NRING: ring slot released by the chain CTA (remote arrival)
-    PB_COUNT = PB_RING_FREE + NRING
+    PB_COUNT
 };
 static_assert(CB_COUNT * 8 <= M_BETA && PB_COUNT * 8 <= M_BETA, "barrier area");
 
@@ -381,17 +380,17 @@ __device__ __forceinline__ uint32_t atom_add_cluster(uint32_t addr, uint32_t v) 
 __device__ __forceinline__ void st_release_cluster(uint32_t addr, uint32_t v) {
     asm volatile("st.release.cluster.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
-__device__ __forceinline__ uint32_t ld_acquire_cta(uint32_t addr) {
+__device__ __forceinline__ uint32_t ld_acquire_remote(uint32_t addr) {
     uint32_t v;
-    asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    asm volatile("ld.acquire.cluster.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
     return v;
 }
-// bounded wait until the u32 at `addr` (this CTA's shared memory) reaches `target`
-__device__ __forceinline__ bool wait_count(uint32_t addr, uint32_t target, volatile uint32_t *abort_flag) {
-    if (ld_acquire_cta(addr) >= target) return true;
+// bounded wait until the u32 at `addr` (another CTA's shared memory) reaches `target`
+__device__ __forceinline__ bool wait_count_remote(uint32_t addr, uint32_t target, volatile uint32_t *abort_flag) {
+    if (ld_acquire_remote(addr) >= target) return true;
     const uint64_t t0 = globaltimer();
     for (;;) {
-        if (ld_acquire_cta(addr) >= target) return true;
+        if (ld_acquire_remote(addr) >= target) return true;
         if (*abort_flag) return false;
         if (globaltimer() - t0 > kWaitLimitNs) {
             *abort_flag = 1;
@@ -400,7 +399,6 @@ __device__ __forceinline__ bool wait_count(uint32_t addr, uint32_t target, volat
         }
     }
 }
-
 __device__ __forceinline__ uint32_t smid() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
@@ -487,6 +485,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint32_t sm = smid();
             *reinterpret_cast<volatile uint32_t *>(miscg + M_SMID) = sm;
             *reinterpret_cast<volatile uint32_t *>(miscg + M_NEXT) = 0u;
+            *reinterpret_cast<volatile uint32_t *>(miscg + M_CONSUMED) = 0u;   // sets pulled so far
             // the shared pool holds a ring per SM id; a launch with one ring per cluster does not
             // index it by SM
             const bool no_ring = !kRingPerCluster && sm >= static_cast<uint32_t>(kMaxRings);
@@ -504,9 +503,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             *reinterpret_cast<volatile uint32_t *>(miscg + M_HTINFO + 16) =
                 (hT_write ? 1u : 0u) | ((transition || p.hT_fp32 != 0) ? 2u : 0u);
         } else {
-            for (int i = 0; i < PB_RING_FREE; ++i) mbar_init(BAR(i), i == PB_STAGE_FULL ? 2 : 1);
-            *reinterpret_cast<volatile uint32_t *>(miscg + M_CONSUMED) = 0u;
-            for (int i = 0; i < NRING; ++i) mbar_init(BAR(PB_RING_FREE + i), 1);
+            for (int i = 0; i < PB_COUNT; ++i) mbar_init(BAR(i), i == PB_STAGE_FULL ? 2 : 1);
             *abort_flag = 0;
         }
         fence_mbar_init();
@@ -577,7 +574,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int n = 0; n < nch; ++n) {
                 const int sl = n & 1, r = n % NRING;
                 if (!wait_bar(BAR(CB_READY + r), (n / NRING) & 1, abort_flag)) break;
+                if (lane == 0) KDA_TRACE_POINT(n, 37);
                 if (n >= 2 && !wait_bar(BAR(CB_SFREE + sl), ((n - 2) >> 1) & 1, abort_flag)) break;
+                if (lane == 0) KDA_TRACE_POINT(n, 38);
                 if (lane == 0) {
                     const unsigned char *src = ring + static_cast<uint64_t>(r) * SET_STRIDE;
                     const uint32_t dst = sbase + CH_SLOT + sl * SET_STRIDE;
@@ -596,13 +595,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int n = 0; n < nch; ++n) {
                 const int sl = n & 1;
                 if (!wait_bar(BAR(CB_FULL + sl), (n >> 1) & 1, abort_flag)) break;
+                if (lane == 0) KDA_TRACE_POINT(n, 39);
                 if (lane == 0) {
-                    if (n + NRING < nch) {
-                        // chunks 0..n have been pulled: any prep CTA may reuse the slot of chunk n
-                        for (uint32_t pr = 1; pr <= static_cast<uint32_t>(NPREP); ++pr)
-                            st_release_cluster(mapa(sbase + PR_MISC + M_CONSUMED, pr), static_cast<uint32_t>(n + 1));
-                    }
                     mbar_arrive(BAR(CB_SFREE + sl));
+                    // chunks 0..n have been pulled: any prep CTA may reuse the slot of chunk n. One
+                    // store into this CTA's own shared memory, which the prep CTAs poll: a release
+                    // store into each of them measured about 0.6 us apiece and held the ring full.
+                    if (n + NRING < nch) st_release_cluster(sbase + CH_MISC + M_CONSUMED, static_cast<uint32_t>(n + 1));
                 }
                 __syncwarp();
             }
@@ -945,7 +944,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
 #endif
                 // the ring slot must have been pulled by the chain CTA (chunk m - NRING)
-                if (m >= NRING && !wait_count(misc + M_CONSUMED, static_cast<uint32_t>(m - NRING + 1), abort_flag))
+                if (m >= NRING && !wait_count_remote(mapa(sbase + CH_MISC + M_CONSUMED, 0),
+                                                     static_cast<uint32_t>(m - NRING + 1), abort_flag))
                     break;
                 if (lane == 0) KDA_TRACE_POINT(m, 18);
                 if (lane == 0) {
