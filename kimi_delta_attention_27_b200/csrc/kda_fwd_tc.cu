@@ -101,7 +101,7 @@ constexpr int NTHREADS = 384;
 #define KDA_NRING 6
 #endif
 constexpr int NRING = KDA_NRING;  // ring slots per cluster (a multiple of NPREP)
-static_assert(NRING % 3 == 0 && NRING >= 6 && NRING <= 15, "ring depth");
+static_assert(NRING % NPREP == 0 && NRING >= 6 && NRING <= 15, "ring depth");
 
 // ---- operand set of one chunk (same byte layout in the global ring and in smem), 128B-swizzled tiles:
 //   Kt^T fp16 [128 key][64 token]              B operand of C3^T (K-major)
