@@ -1441,10 +1441,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         float x[16];
 #pragma unroll
                         for (int r = 0; r < 16; ++r) x[r] = r == li ? 1.f : 0.f;
+                        // A is read four columns at a time (one 16-byte broadcast load per row and
+                        // column group) just before the group's four steps
 #pragma unroll
-                        for (int j = 0; j < 15; ++j)
+                        for (int g = 0; g < 4; ++g) {
+                            float4 a4[16];
 #pragma unroll
-                            for (int r = j + 1; r < 16; ++r) x[r] = fmaf(-Ab[r * AKK_LD + j], x[j], x[r]);
+                            for (int r = 4 * g + 1; r < 16; ++r)
+                                a4[r] = *reinterpret_cast<const float4 *>(Ab + r * AKK_LD + 4 * g);
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj) {
+                                const int j = 4 * g + jj;
+#pragma unroll
+                                for (int r = j + 1; r < 16; ++r) {
+                                    const float a = jj == 0 ? a4[r].x : jj == 1 ? a4[r].y : jj == 2 ? a4[r].z : a4[r].w;
+                                    x[r] = fmaf(-a, x[j], x[r]);
+                                }
+                            }
+                        }
 #pragma unroll
                         for (int r = 0; r < 16; ++r) T[(16 * wb + r) * AKK_LD + 16 * wb + li] = x[r];
                     }
