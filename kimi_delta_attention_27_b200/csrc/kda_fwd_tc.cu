@@ -167,7 +167,8 @@ enum {
 };
 // prep barriers
 enum {
-    PB_STAGE_FULL = 0, PB_STAGE_FREE, PB_VSTAGE_FULL, PB_VSTAGE_FREE, PB_SPARE4,
+    PB_STAGE_FULL = 0, PB_STAGE_FREE, PB_VSTAGE_FULL, PB_VSTAGE_FREE,
+    PB_STAGE_RAW,       // tx: the tiles of a partial chunk, before the loader zeroes its tail rows
     PB_P1_DONE, PB_SPARE6,
     PB_WAV_DONE, PB_SPARE8, PB_SPARE9,
     PB_OUTA_READY,      // Kt^T final (over Kc^T)
@@ -857,6 +858,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // each local chunk kk: the chunk index (queue of 4), its beta (queue of 2), q, k, g by
             // TMA, then v.
             volatile uint32_t *chunkq = reinterpret_cast<volatile uint32_t *>(miscg + M_CHUNKQ);
+            uint32_t nraw = 0;   // partial chunks staged so far (phases of PB_STAGE_RAW)
             for (int kk = 0;; ++kk) {
                 if (kk >= 1 && !wait_bar(BAR(PB_STAGE_FREE), (kk - 1) & 1, abort_flag)) break;
                 uint32_t mm = 0;
@@ -875,17 +877,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 const int64_t t0 = bos + static_cast<int64_t>(m) * C;
                 const int32_t row = static_cast<int32_t>(t0);
+                // a partial chunk lands on its own barrier first: this warp zeroes the staged rows
+                // past the sequence's end (the next sequence's tokens, or TMA fill) before handing
+                // the tiles over, so that S1 needs no row masks
+                const int Lz = static_cast<int>(eos - t0 < C ? eos - t0 : C);
+                const uint32_t land = Lz < C ? BAR(PB_STAGE_RAW) : BAR(PB_STAGE_FULL);
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(BAR(PB_STAGE_FULL), kGate == kGateF32    ? STAGE_TX
-                                                              : kGate == kGateBF16 ? STAGE_TX - 16384u
-                                                                                   : STAGE_TX - 32768u);
-                    tma_load_3d(sbase + PR_STG + STG_Q, &maps.q, BAR(PB_STAGE_FULL), 0, h, row);
-                    tma_load_3d(sbase + PR_STG + STG_K, &maps.k, BAR(PB_STAGE_FULL), 0, h, row);
+                    mbar_arrive_expect_tx(land, kGate == kGateF32    ? STAGE_TX
+                                                : kGate == kGateBF16 ? STAGE_TX - 16384u
+                                                                     : STAGE_TX - 32768u);
+                    tma_load_3d(sbase + PR_STG + STG_Q, &maps.q, land, 0, h, row);
+                    tma_load_3d(sbase + PR_STG + STG_K, &maps.k, land, 0, h, row);
                     // a bf16 gate tile goes to the upper half of the fp32 one's place
                     if constexpr (kGate == kGateF32)
-                        tma_load_3d(sbase + PR_STG + STG_G, &maps.g, BAR(PB_STAGE_FULL), 0, h, row);
+                        tma_load_3d(sbase + PR_STG + STG_G, &maps.g, land, 0, h, row);
                     else if constexpr (kGate == kGateBF16)
-                        tma_load_3d(sbase + PR_STG + STG_G + 16384, &maps.g, BAR(PB_STAGE_FULL), 0, h, row);
+                        tma_load_3d(sbase + PR_STG + STG_G + 16384, &maps.g, land, 0, h, row);
                 }
                 float *betaq = reinterpret_cast<float *>(miscg + M_BETAQ) + (kk & 1) * C;
                 for (int i = lane; i < C; i += 32) {
@@ -902,6 +909,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         if ((p.flags & kFlagGateLogsigmoid) && tok < eos) x = log2_sigmoid(x) * kLn2;
                         gq[i] = x;
                     }
+                }
+                if (Lz < C) {
+                    if (!wait_bar(BAR(PB_STAGE_RAW), nraw & 1u, abort_flag)) break;
+                    ++nraw;
+                    for (int e = lane; e < (C - Lz) * 16; e += 32) {
+                        const uint32_t off = static_cast<uint32_t>((Lz + (e >> 4)) * 256 + (e & 15) * 16);
+                        st_shared_v4(sbase + PR_STG + STG_Q + off, 0u, 0u, 0u, 0u);
+                        st_shared_v4(sbase + PR_STG + STG_K + off, 0u, 0u, 0u, 0u);
+                    }
+                    if constexpr (kGate == kGateF32) {
+                        for (int e = lane; e < (C - Lz) * 32; e += 32)
+                            st_shared_v4(sbase + PR_STG + STG_G + static_cast<uint32_t>((Lz + (e >> 5)) * 512 + (e & 31) * 16),
+                                         0u, 0u, 0u, 0u);
+                    } else if constexpr (kGate == kGateBF16) {
+                        for (int e = lane; e < (C - Lz) * 16; e += 32)
+                            st_shared_v4(sbase + PR_STG + STG_G + 16384 +
+                                             static_cast<uint32_t>((Lz + (e >> 4)) * 256 + (e & 15) * 16),
+                                         0u, 0u, 0u, 0u);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(BAR(PB_STAGE_FULL));   // first arrival: the zeroed tiles
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(BAR(PB_STAGE_FULL));   // second arrival: index and beta stored
@@ -1024,35 +1052,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const unsigned long long trace_sfull = globaltimer();
 #endif
                 const int m = static_cast<int>(chunkq[kk & 3]);   // this CTA's kk-th chunk
+                // past the last chunk the phase below still runs up to its first barrier (on stale
+                // tiles, which is harmless), and every warp leaves there together
                 const bool no_chunk = m >= nch;
-                if (!no_chunk) {
-                    // partial chunk: the staged rows past the sequence's end hold the next
-                    // sequence's tokens (or TMA fill); zero them so that S1 needs no row masks
-                    const int64_t tz = bos + static_cast<int64_t>(m) * C;
-                    const int Lz = static_cast<int>(eos - tz < C ? eos - tz : C);
-                    if (Lz < C) {
-                        for (int e = t; e < (C - Lz) * 16; e += 256) {
-                            const uint32_t off = static_cast<uint32_t>((Lz + (e >> 4)) * 256 + (e & 15) * 16);
-                            st_shared_v4(sbase + PR_STG + STG_Q + off, 0u, 0u, 0u, 0u);
-                            st_shared_v4(sbase + PR_STG + STG_K + off, 0u, 0u, 0u, 0u);
-                        }
-                        if constexpr (kGate == kGateF32) {
-                            for (int e = t; e < (C - Lz) * 32; e += 256)
-                                st_shared_v4(sbase + PR_STG + STG_G +
-                                                 static_cast<uint32_t>((Lz + (e >> 5)) * 512 + (e & 31) * 16),
-                                             0u, 0u, 0u, 0u);
-                        } else if constexpr (kGate == kGateBF16) {
-                            for (int e = t; e < (C - Lz) * 16; e += 256)
-                                st_shared_v4(sbase + PR_STG + STG_G + 16384 +
-                                                 static_cast<uint32_t>((Lz + (e >> 4)) * 256 + (e & 15) * 16),
-                                             0u, 0u, 0u, 0u);
-                        }
-                    }
-                }
-                if (named_bar_any(2, 256, no_chunk || *abort_flag != 0)) {
-                    if (t == 0) mbar_arrive(BAR(PB_OUTA_READY));   // the publisher's end signal
-                    break;
-                }
                 // rows of this chunk that hold tokens (the others are zero in the staging tiles)
                 const int Lrows = static_cast<int>(eos - (bos + static_cast<int64_t>(m) * C) < C
                                                        ? eos - (bos + static_cast<int64_t>(m) * C)
@@ -1156,8 +1158,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     // quarter decays beyond the single anchor's range" with the abort flag; only when
                     // that is set does a second barrier tell the two apart
                     const bool unsafe = !(qsum.x >= -kQuarterRangeLog2) || !(qsum.y >= -kQuarterRangeLog2);
-                    if (__builtin_expect(named_bar_any(2, 256, unsafe || *abort_flag != 0), 0)) {
-                        if (named_bar_any(2, 256, *abort_flag != 0)) break;
+                    if (__builtin_expect(named_bar_any(2, 256, unsafe || no_chunk || *abort_flag != 0), 0)) {
+                        if (named_bar_any(2, 256, no_chunk || *abort_flag != 0)) {
+                            if (t == 0) mbar_arrive(BAR(PB_OUTA_READY));   // the publisher's end signal
+                            break;
+                        }
                         robust = true;
                         // the sub-block path floors the gates: again with the floored sums
                         sp[0] = sp[1] = make_float2(0.f, 0.f);
