@@ -126,6 +126,32 @@ __device__ __forceinline__ Unit unit_of(const BwdParams &p) {
     return u;
 }
 
+__device__ __forceinline__ void prefetch_l2(const void *ptr) { asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr)); }
+
+// Ask L2 for the inputs of the chunk at t0 (the next one this CTA loads), one request per 128-byte
+// line of its rows: the chunks run in a sequential order, so the loads of each one would otherwise
+// wait on HBM latency in full.
+__device__ void prefetch_chunk(const BwdParams &p, const Unit &u, int64_t t0, bool with_do) {
+    const int t = threadIdx.x;
+    if (t0 < u.bos || t0 >= u.eos) return;
+    const int L = static_cast<int>(u.eos - t0 < CB ? u.eos - t0 : CB);
+    const int H = p.num_heads;
+    const int r = t >> 4, part = t & 15;
+    if (r >= L) return;
+    const size_t row = (static_cast<size_t>(t0) + r) * H + u.h;
+    if (part < 2) {                          // k and q rows: 256 bytes each
+        prefetch_l2(p.k + row * D + part * 64);
+        prefetch_l2(p.q + row * D + part * 64);
+    } else if (part < 6) {                   // g rows: 512 bytes
+        prefetch_l2(p.g + row * D + (part - 2) * 32);
+    } else if (part == 6) {                  // this CTA's value slice of v and dO: 64 bytes
+        prefetch_l2(p.v + row * D + u.vs * VS);
+        if (with_do) prefetch_l2(p.dout + row * D + u.vs * VS);
+    } else if (part == 7) {
+        prefetch_l2(p.beta + row);
+    }
+}
+
 // Load chunk n of the unit (rows past the end are zero, with no decay) and form its factors:
 // G (floored, log2 units), Kd, Qd, Kt, the anchored Kl, Ql, Kr, e^Gl, beta, and the V and dO
 // slices (dO only when `with_do`).
@@ -340,6 +366,7 @@ __global__ void __launch_bounds__(NT, 1) kda_bwd_kernel(const BwdParams p) {
             const int64_t t0 = u.bos + static_cast<int64_t>(gi) * GRP + sub * CB;
             if (t0 >= u.eos) break;
             const int L = static_cast<int>(u.eos - t0 < CB ? u.eos - t0 : CB);
+            prefetch_chunk(p, u, t0 + CB, false);
             load_chunk(p, u, t0, L, false, sm);
             chunk_blocks(sm);
             chunk_xd(sm, S);
@@ -368,6 +395,7 @@ __global__ void __launch_bounds__(NT, 1) kda_bwd_kernel(const BwdParams p) {
         for (int sub = 0; sub + 1 < nsub; ++sub) {
             const int64_t t0 = g0 + sub * CB;
             const int L = static_cast<int>(u.eos - t0 < CB ? u.eos - t0 : CB);
+            prefetch_chunk(p, u, t0 + CB, sub + 2 == nsub);   // the last one is next taken backwards
             load_chunk(p, u, t0, L, false, sm);
             chunk_blocks(sm);
             chunk_xd(sm, sm + SM_SCK + sub * D * VP);
@@ -377,6 +405,13 @@ __global__ void __launch_bounds__(NT, 1) kda_bwd_kernel(const BwdParams p) {
             const int64_t t0 = g0 + sub * CB;
             const int L = static_cast<int>(u.eos - t0 < CB ? u.eos - t0 : CB);
             const float *S0 = sm + SM_SCK + sub * D * VP;
+            if (sub > 0) {
+                prefetch_chunk(p, u, t0 - CB, true);
+            } else if (gi > 0) {
+                // the next group: its checkpoint, then its first chunk
+                if (t < D) prefetch_l2(state_at(p.workspace, u.slot0 + gi - 1) + static_cast<size_t>(t) * D);
+                prefetch_chunk(p, u, g0 - GRP, false);   // a full group: recomputed forwards first
+            }
             load_chunk(p, u, t0, L, true, sm);
             chunk_blocks(sm);
             chunk_xd(sm, S0);
