@@ -172,10 +172,10 @@ enum {
     PB_P1_DONE, PB_SPARE6,
     PB_WAV_DONE, PB_SPARE8, PB_SPARE9,
     PB_OUTA_READY,      // Kt^T final (over Kc^T)
-    PB_OUTB_READY,      // -W^T final (over the fp32 T workspace)
-    PB_OUTC_READY,      // Qd^T (over A), T' and Aqk, V, e^Gl final
+    PB_OUTB_READY,      // -W^T (over the fp32 T workspace) and Qd^T (over A) final
+    PB_OUTC_READY,      // T' and Aqk, e^Gl final (after the solve)
     PB_OUTA_FREE,       // publisher has read part A out
-    PB_OUTC_FREE,       // publisher has read part C out
+    PB_OUTC_FREE,       // publisher has read parts C and B out
     PB_COUNT
 };
 static_assert(CB_COUNT * 8 <= M_BETA && PB_COUNT * 8 <= M_BETA, "barrier area");
@@ -986,23 +986,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     mbar_arrive(BAR(PB_VSTAGE_FREE));   // the next value tile may be loaded
                 }
                 __syncwarp();
-                if (!wait_bar(BAR(PB_OUTB_READY), kk & 1, abort_flag)) break;
-                if (lane == 0) {
-                    KDA_TRACE_POINT(m, 20);
-                    bulk_s2g(set + SET_W, sbase + PR_T, 16384);
-                    bulk_commit();
-                    KDA_TRACE_POINT(m, 21);
-                }
-                __syncwarp();
+                // part C, final once the solve is done: it is on its way while W' runs, so that
+                // only part B is left to write when the chunk ends
                 if (!wait_bar(BAR(PB_OUTC_READY), kk & 1, abort_flag)) break;
                 if (lane == 0) {
-                    KDA_TRACE_POINT(m, 22);
-                    bulk_s2g(set + SET_Q, sbase + PR_AKK, 16384);
+                    KDA_TRACE_POINT(m, 20);
                     bulk_s2g(set + SET_T, sbase + PR_AVT, 8192);
                     bulk_s2g(set + SET_AQK, sbase + PR_AVT + 8192, 8192);
                     bulk_s2g(set + SET_DEC, misc + M_DEC + (kk & 1) * 512, 512);
                     bulk_commit();
-                    bulk_wait_read0();
+                    KDA_TRACE_POINT(m, 21);
+                }
+                __syncwarp();
+                if (!wait_bar(BAR(PB_OUTB_READY), kk & 1, abort_flag)) break;
+                if (lane == 0) {
+                    KDA_TRACE_POINT(m, 22);
+                    bulk_s2g(set + SET_W, sbase + PR_T, 16384);
+                    bulk_s2g(set + SET_Q, sbase + PR_AKK, 16384);
+                    bulk_commit();
+                    bulk_wait_read0();   // parts C and B read out
                     KDA_TRACE_POINT(m, 23);
                     mbar_arrive(BAR(PB_OUTC_FREE));
                     bulk_wait0();
@@ -1643,6 +1645,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 fence_proxy_async_smem();
                 if (t == 0) KDA_TRACE_POINT(m, 17);
                 if (named_bar_any(2, 256, *abort_flag != 0)) break;
+                if (t == 0) mbar_arrive(BAR(PB_OUTC_READY));   // T', Aqk and e^Gl are final
                 if (warp == 4) {
                     tc_fence_after();
                     if (elect_one()) {
@@ -1695,7 +1698,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (named_bar_any(2, 256, *abort_flag != 0)) break;
                 if (t == 0) {
                     mbar_arrive(BAR(PB_OUTB_READY));
-                    mbar_arrive(BAR(PB_OUTC_READY));
                     KDA_TRACE_POINT(m, 6);
                 }
             }
